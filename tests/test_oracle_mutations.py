@@ -1,0 +1,63 @@
+"""The pins have teeth: each plausible slip, planted in a copy of the oracle's
+C source and compiled on the CPU, must make at least one pin test fail."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "bra_oracle.c")
+
+# (name, original text, mutated text)
+MUTATIONS = [
+    ("no_softmax_scale", "double scale = 1.0 / sqrt((double)d);", "double scale = 1.0;"),
+    ("pool_sum_not_mean", "= sum / (double)n;", "= sum;"),
+    ("affinity_transposed",
+     "a[((size_t)bh * R + r) * R + s] = dot;", "a[((size_t)bh * R + s) * R + r] = dot;"),
+    ("tie_to_higher_index",
+     "return (a->index > b->index) - (a->index < b->index);",
+     "return (a->index < b->index) - (a->index > b->index);"),
+    ("topk_smallest_first", "if (a->value > b->value) return -1;", "if (a->value < b->value) return -1;"),
+    ("region_column_major", "int ri = r / S, rj = r % S;", "int ri = r % S, rj = r / S;"),
+    ("token_column_major", "*y = ri * hs + t / ws;", "*y = ri * hs + t % hs;"),
+    ("softmax_weights_perturbed", "s[j] = exp(s[j] - mx);", "s[j] = exp(s[j] - mx + 1e-3 * j);"),
+    ("values_from_keys", "num += s[j] * v[key_off[j] + c];", "num += s[j] * k[key_off[j] + c];"),
+    ("first_route_only", "int rr = route[m];", "int rr = route[0];"),
+]
+
+
+def build_variant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation {name}: anchor text not found exactly once"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"lib{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", str(lib), str(path), "-lm"])
+    return str(lib)
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(tmp_path, name, old, new):
+    import test_oracle_pins as pins
+    lib = build_variant(tmp_path, name, old, new)
+    checks = [
+        pins.test_region_pool_is_block_mean,
+        pins.test_affinity_equals_average_token_affinity,
+        pins.test_affinity_is_not_scaled_and_not_transposed,
+        lambda: pins.test_topk_matches_subset_enumeration(7, True),
+        pins.test_topk_duplicate_region_lower_index_first,
+        lambda: pins.test_full_topk_is_dense_attention(2),
+        lambda: pins.test_gather_equals_region_masked_dense((1, 12, 8, 6, 3, 4, 3)),
+        pins.test_worked_example_by_hand,
+        pins.test_region_permutation_equivariance,
+        lambda: pins.test_brute_force_tiny(2, 2),
+    ]
+    failures = 0
+    with oracle.swapped_library(lib):
+        for check in checks:
+            try:
+                check()
+            except (AssertionError, ValueError):
+                failures += 1
+    assert failures > 0, f"no pin caught mutation {name}"
