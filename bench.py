@@ -1,0 +1,378 @@
+"""Benchmark of the Bi-Level Routing Attention forward on B200.
+
+One step = one pass of the whole path (region pooling, routing, token
+attention) over one batch of the BiFormer stage-1 workload: B=64, 56x56 map,
+C=64, 2 heads of 32, S=7 (49 regions of 8x8 tokens), topk=1, bf16, seeded
+synthetic inputs.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU, each rank an
+independent replica on its own batch (the path has no exchange step), and
+the value is all ranks' tokens over the slowest rank's device time.
+
+``--impl reference`` times the float64 CPU oracle on bounded samples of the
+same workload (the comparison arm; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import bra_inputs as bi  # noqa: E402
+
+WORKLOAD = "stage1"
+METRIC = "BRA forward tokens/s on 1 B200 (bf16) and % of tensor/HBM roofline"
+L2_BYTES = 126 * 2**20
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM bytes per launch of the attention kernel on the stage-1 workload, from
+# an ncu capture, keyed by the sha256 of the kernel sources it was taken on;
+# reported as ``traffic`` only while the sources are unchanged.
+TRAFFIC_RECORDS: dict[str, float] = {}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=500)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=WORKLOAD, choices=list(bi.WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=20)
+    return p.parse_args()
+
+
+def workload_config(shape: bi.BraShape, name: str) -> dict:
+    return {"workload": f"{name}: B{shape.B} {shape.H}x{shape.W} C{shape.C} heads{shape.heads} "
+                        f"d{shape.d} S{shape.S} topk{shape.topk} {shape.dtype}",
+            "B": shape.B, "H": shape.H, "W": shape.W, "C": shape.C, "heads": shape.heads,
+            "S": shape.S, "topk": shape.topk, "tokens_per_step": shape.tokens}
+
+
+def byte_counts(shape: bi.BraShape) -> dict:
+    es = 2 if shape.dtype == "bf16" else 4
+    m = shape.tokens * shape.C * es
+    idx = shape.B * shape.heads * shape.R * shape.topk * 4
+    means = shape.B * shape.heads * shape.R * shape.d * 4
+    return {
+        "map": m,
+        "idx": idx,
+        # minimal bytes of the whole path: Q, K, V read once, O and I^r written once
+        "path_min": 4 * m + idx,
+        # attention kernel: Q, K, V read, O written, I^r read
+        "attend": 4 * m + idx,
+        # pooling kernel: Q, K read, means written
+        "pool": 2 * m + 2 * means,
+    }
+
+
+def attention_flops(shape: bi.BraShape) -> float:
+    # QK^T and PV: 2 matmuls x (tokens x topk*n keys x C) multiply-adds x 2 flop
+    return 4.0 * shape.tokens * shape.topk * shape.n * shape.C
+
+
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dynamic_sparse_attention_bra_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("attend") or name in ("common.cuh", "kernels.h"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples: list[int] = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report what we could not sample
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def report(self) -> dict:
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
+                          batches_per_call: int | None = None) -> dict:
+    """The float64 oracle (single thread) on bounded samples of the workload."""
+    import oracle
+    inp = bi.make_inputs(shape, seed)
+    bpc = batches_per_call or shape.B
+    tokens = 0
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        b0 = (calls * bpc) % shape.B
+        sl = slice(b0, b0 + bpc)
+        oracle.bra_forward(inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl], shape.heads, shape.S, shape.topk)
+        tokens += bpc * shape.H * shape.W
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": tokens / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{calls} oracle calls of {bpc} of {shape.B} images ({tokens} tokens) "
+                      f"in {el:.1f} s, float64, one thread"}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    shape, seed = bi.WORKLOADS[args.workload]
+    import oracle
+    inp = bi.make_inputs(shape, seed)
+    bpc = 1  # one image per step: a bounded sample of the batch
+    step = lambda i: oracle.bra_forward(inp.q_f64[i % shape.B:i % shape.B + bpc],
+                                        inp.k_f64[i % shape.B:i % shape.B + bpc],
+                                        inp.v_f64[i % shape.B:i % shape.B + bpc],
+                                        shape.heads, shape.S, shape.topk)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    tokens = args.steps * bpc * shape.H * shape.W
+    value = tokens / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**workload_config(shape, args.workload), "sample_images_per_step": bpc},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{bpc} of {shape.B} images per step, float64 oracle, one thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    shape, seed = bi.WORKLOADS[args.workload]
+    inp = bi.make_inputs(shape, seed + 1000 * rank)
+    es = 2 if shape.dtype == "bf16" else 4
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+    def host(x):
+        t = torch.from_numpy(x)
+        return t.view(torch.bfloat16) if shape.dtype == "bf16" else t
+
+    host_qkv = [host(a).pin_memory() for a in (inp.q_store, inp.k_store, inp.v_store)]
+    cnt = byte_counts(shape)
+    set_bytes = 4 * cnt["map"] + cnt["idx"]
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    sets = []
+    for _ in range(nsets):
+        q, k, v = (h.to(dev) for h in host_qkv)
+        sets.append(dict(
+            q=q, k=k, v=v, o=torch.empty_like(q),
+            idx=torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device=dev),
+            ws=torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device=dev)))
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+
+    def step(i):
+        b = sets[i % nsets]
+        bra.bra_route(s, b["q"], b["k"], b["idx"], b["ws"], sp)
+        bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+
+    # Timed region: K steps; events around each attention launch on the same
+    # stream give the attention kernel's own average duration.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(args.steps):
+                b = sets[i % nsets]
+                bra.bra_route(s, b["q"], b["k"], b["idx"], b["ws"], sp)
+                ev[i][0].record(stream)
+                bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
+                ev[i][1].record(stream)
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    attend_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    for b in sets:
+        st = bra.bra_device_status(s, b["ws"], sp)
+        if st != bra.BRA_OK:
+            raise RuntimeError(f"device status after timing: {bra.bra_status_string(st)}")
+
+    # End to end through the public API with host buffers: pinned Q, K, V in,
+    # O and I^r out, every step, copies inside the timed region.
+    o_host = torch.empty(host_qkv[0].shape, dtype=tdt).pin_memory()
+    idx_host = torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32).pin_memory()
+    b0 = sets[0]
+    h2d = 3 * cnt["map"]
+    d2h = cnt["map"] + cnt["idx"]
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for dst, src in zip((b0["q"], b0["k"], b0["v"]), host_qkv):
+                dst.copy_(src, non_blocking=True)
+            bra.bra_forward(s, b0["q"], b0["k"], b0["v"], b0["o"], b0["idx"], b0["ws"], sp)
+            o_host.copy_(b0["o"], non_blocking=True)
+            idx_host.copy_(b0["idx"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+
+    times = torch.tensor([total_ms, attend_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    total_ms, attend_ms, e2e_ms = times.tolist()
+    ms_per_step = total_ms / args.steps
+    tokens = shape.tokens * world
+    value = tokens / (ms_per_step * 1e-3)
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        achieved = cnt["attend"] / (attend_ms * 1e-3) / 1e9
+        digest = kernel_sources_hash()
+        traffic = TRAFFIC_RECORDS.get(digest)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": shape.dtype, "data": "synthetic",
+            "config": {**workload_config(shape, args.workload), "parallelism": f"replicas{world}",
+                       "l2": f"rotating {nsets} input sets ({nsets * set_bytes / 2**20:.0f} MiB) > 126 MiB L2"},
+            "roofline": {
+                "kernel": "bra_attend", "bound": "hbm", "achieved": achieved, "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                "algorithmic_bytes": cnt["attend"], "launch_ms": attend_ms,
+            },
+            "path_roofline": {
+                "min_bytes": cnt["path_min"], "flops": attention_flops(shape),
+                "time_us": ms_per_step * 1e3,
+                "frac": cnt["path_min"] / peak / 1e9 / (ms_per_step * 1e-3),
+            },
+            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.report(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_throughput(shape, seed)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

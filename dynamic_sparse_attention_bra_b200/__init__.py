@@ -1,0 +1,153 @@
+"""Bi-Level Routing Attention (BiFormer) forward on B200, sm_100a.
+
+A thin ctypes binding over the C ABI of ``libbra_b200.so`` (declared in
+``include/bra.h``).  Every step of the path runs in the library's CUDA
+kernels; this module only turns torch tensors into pointers and sizes and
+turns status codes into exceptions.  There is no CPU fallback: if the
+library is missing the import of the binding fails.
+
+Entry points (same names as the C ABI):
+
+    bra_workspace_bytes(shape)
+    bra_route(shape, q, k, idx, workspace, stream=None)
+    bra_attend(shape, q, k, v, idx, o, workspace, stream=None)
+    bra_forward(shape, q, k, v, o, idx, workspace, stream=None)
+    bra_device_status(shape, workspace, stream=None)
+
+and a convenience wrapper ``forward(q, k, v, heads, S, topk)`` that
+allocates the outputs and workspace with torch and returns ``(o, idx)``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
+    "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libbra_b200.so")
+
+BRA_OK, BRA_ERR_INVALID_ARG, BRA_ERR_UNSUPPORTED, BRA_ERR_CUDA, BRA_ERR_TIMEOUT, BRA_ERR_BAD_ROUTE = range(6)
+BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
+
+EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
+                    "bra_device_status", "bra_status_string", "bra_version")
+
+
+class BraShape(ctypes.Structure):
+    """Mirror of ``bra_shape``."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("C", ctypes.c_int),
+                ("heads", ctypes.c_int), ("S", ctypes.c_int), ("topk", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class BraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {bra_status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(library_path):
+        raise ImportError(
+            f"{library_path} is not built; run `python -m dynamic_sparse_attention_bra_b200.build`")
+    lib = ctypes.CDLL(library_path)
+    vp, sp = ctypes.c_void_p, ctypes.POINTER(BraShape)
+    lib.bra_workspace_bytes.argtypes = [sp]
+    lib.bra_workspace_bytes.restype = ctypes.c_size_t
+    lib.bra_route.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.bra_attend.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
+    lib.bra_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
+    lib.bra_device_status.argtypes = [sp, vp, vp]
+    for f in (lib.bra_route, lib.bra_attend, lib.bra_forward, lib.bra_device_status):
+        f.restype = ctypes.c_int
+    lib.bra_status_string.argtypes = [ctypes.c_int]
+    lib.bra_status_string.restype = ctypes.c_char_p
+    lib.bra_version.argtypes = []
+    lib.bra_version.restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def bra_status_string(status: int) -> str:
+    return _lib.bra_status_string(status).decode()
+
+
+def shape_for(B: int, H: int, W: int, C: int, heads: int, S: int, topk: int, dtype) -> BraShape:
+    """``bra_shape`` for a problem; ``dtype`` is a torch dtype or "f32"/"bf16"."""
+    name = str(dtype)
+    code = BRA_DTYPE_BF16 if "bf16" in name or "bfloat16" in name else BRA_DTYPE_F32
+    return BraShape(B, H, W, C, heads, S, topk, code)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != BRA_OK:
+        raise BraError(status, where)
+
+
+def bra_workspace_bytes(shape: BraShape) -> int:
+    return int(_lib.bra_workspace_bytes(ctypes.byref(shape)))
+
+
+def bra_route(shape: BraShape, q, k, idx, workspace, stream=None) -> None:
+    _check(_lib.bra_route(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(idx), _ptr(workspace),
+                          _stream(stream)), "bra_route")
+
+
+def bra_attend(shape: BraShape, q, k, v, idx, o, workspace, stream=None) -> None:
+    _check(_lib.bra_attend(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
+                           _ptr(workspace), _stream(stream)), "bra_attend")
+
+
+def bra_forward(shape: BraShape, q, k, v, o, idx, workspace, stream=None) -> None:
+    _check(_lib.bra_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(idx),
+                            _ptr(workspace), _stream(stream)), "bra_forward")
+
+
+def bra_device_status(shape: BraShape, workspace, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device status code."""
+    return int(_lib.bra_device_status(ctypes.byref(shape), _ptr(workspace), _stream(stream)))
+
+
+def _check_tensor(t, name: str, dtype, numel: int):
+    import torch
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous() and t.dtype == dtype
+            and t.numel() == numel):
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor of {numel} elements")
+
+
+def forward(q, k, v, heads: int, S: int, topk: int, stream=None):
+    """O, I^r for channels-last q, k, v [B, H, W, C] (float32 or bfloat16).
+
+    Allocates O [B, H, W, C], I^r int32 [B, heads, S*S, topk] and a zeroed
+    workspace with torch on q's device, then runs ``bra_forward``."""
+    import torch
+    B, H, W, C = q.shape
+    shape = shape_for(B, H, W, C, heads, S, topk, q.dtype)
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, name, q.dtype, B * H * W * C)
+    nbytes = bra_workspace_bytes(shape)
+    if nbytes == 0:
+        raise BraError(BRA_ERR_INVALID_ARG, "forward")
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    idx = torch.empty((B, heads, S * S, topk), dtype=torch.int32, device=q.device)
+    bra_forward(shape, q, k, v, o, idx, ws, stream)
+    return o, idx

@@ -1,0 +1,16 @@
+// Tensor-core (tcgen05) token attention for bf16, head dim 32 (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "../../include/bra.h"
+#include "common.cuh"
+
+namespace bra {
+
+// Launches the tcgen05 attention for ``g`` when it covers the shape; returns
+// BRA_ERR_UNSUPPORTED (and launches nothing) when it does not.
+bra_status attend_tc_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                            const int32_t* idx, void* o, int* status, cudaStream_t stream);
+
+}  // namespace bra

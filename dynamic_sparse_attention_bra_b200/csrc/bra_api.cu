@@ -1,0 +1,175 @@
+// C ABI of the BRA library: argument checks, workspace layout and launches.
+// Declarations and the contract of every entry point are in include/bra.h.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/bra.h"
+#include "attend_tc.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bra {
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t elem_bytes(int dtype) { return dtype == BRA_DTYPE_BF16 ? 2 : 4; }
+
+// Checks ``s``; fills ``g``.  BRA_OK, BRA_ERR_INVALID_ARG or BRA_ERR_UNSUPPORTED.
+bra_status make_geometry(const bra_shape* s, Geometry* g) {
+    if (!s) return BRA_ERR_INVALID_ARG;
+    if (s->B < 0 || s->H <= 0 || s->W <= 0 || s->C <= 0 || s->heads <= 0 || s->S <= 0)
+        return BRA_ERR_INVALID_ARG;
+    if (s->H % s->S || s->W % s->S || s->C % s->heads) return BRA_ERR_INVALID_ARG;
+    if (s->S > 65535 / s->S || s->topk < 1 || s->topk > s->S * s->S) return BRA_ERR_INVALID_ARG;
+    if (s->dtype != BRA_DTYPE_F32 && s->dtype != BRA_DTYPE_BF16) return BRA_ERR_INVALID_ARG;
+    // All index arithmetic inside the kernels is 64-bit from the token offset
+    // up; per-dimension sizes must still fit the grid.
+    if ((int64_t)s->H * s->W > (int64_t)1 << 30 || s->B > 65535) return BRA_ERR_UNSUPPORTED;
+    g->B = s->B; g->H = s->H; g->W = s->W; g->C = s->C; g->heads = s->heads; g->S = s->S;
+    g->topk = s->topk;
+    g->d = s->C / s->heads;
+    g->R = s->S * s->S;
+    g->hs = s->H / s->S;
+    g->ws = s->W / s->S;
+    g->n = g->hs * g->ws;
+    if (g->d != 32) return BRA_ERR_UNSUPPORTED;
+    if (g->R > kMaxRegions) return BRA_ERR_UNSUPPORTED;
+    if (s->heads > 65535) return BRA_ERR_UNSUPPORTED;
+    // pool: one 16-byte vector column per thread must cover C
+    if ((size_t)s->C * elem_bytes(s->dtype) > 16u * kPoolThreads) return BRA_ERR_UNSUPPORTED;
+    return BRA_OK;
+}
+
+size_t means_bytes(const Geometry& g) {
+    return round_up((size_t)g.B * g.heads * g.R * g.d * sizeof(float), 256);
+}
+
+struct Workspace {
+    float* qr;
+    float* kr;
+    int* status;
+};
+
+Workspace carve(const Geometry& g, void* ws) {
+    char* base = static_cast<char*>(ws);
+    const size_t mb = means_bytes(g);
+    return {reinterpret_cast<float*>(base), reinterpret_cast<float*>(base + mb),
+            reinterpret_cast<int*>(base + 2 * mb)};
+}
+
+bra_status route_impl(const bra_shape* s, const Geometry& g, const void* q, const void* k,
+                      int32_t* idx, const Workspace& w, cudaStream_t st) {
+    if (g.B == 0) return BRA_OK;
+    const bool bf16 = s->dtype == BRA_DTYPE_BF16;
+    if (launch_pool(bf16, q, k, w.qr, w.kr, g, st) != cudaSuccess) return BRA_ERR_CUDA;
+    if (launch_route(w.qr, w.kr, idx, g, st) != cudaSuccess) return BRA_ERR_CUDA;
+    return BRA_OK;
+}
+
+bra_status attend_impl(const bra_shape* s, const Geometry& g, const void* q, const void* k,
+                       const void* v, const int32_t* idx, void* o, const Workspace& w,
+                       cudaStream_t st) {
+    if (g.B == 0) return BRA_OK;
+    const bool bf16 = s->dtype == BRA_DTYPE_BF16;
+    if (bf16) {
+        const bra_status tc = attend_tc_launch(g, q, k, v, idx, o, w.status, st);
+        if (tc != BRA_ERR_UNSUPPORTED) return tc;
+    }
+    if ((int64_t)g.R * simt_plan(g).chunks > 0x7fffffff) return BRA_ERR_UNSUPPORTED;
+    if (launch_attend_simt(bf16, q, k, v, idx, o, g, w.status, st) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    return BRA_OK;
+}
+
+}  // namespace
+}  // namespace bra
+
+using namespace bra;
+
+extern "C" {
+
+size_t bra_workspace_bytes(const bra_shape* shape) {
+    Geometry g;
+    if (make_geometry(shape, &g) != BRA_OK) return 0;
+    return 2 * means_bytes(g) + kStatusBytes;
+}
+
+bra_status bra_route(const bra_shape* shape, const void* q, const void* k, int32_t* idx,
+                     void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!q || !k || !idx || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(idx) || !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    return route_impl(shape, g, q, k, idx, carve(g, workspace), static_cast<cudaStream_t>(stream));
+}
+
+bra_status bra_attend(const bra_shape* shape, const void* q, const void* k, const void* v,
+                      const int32_t* idx, void* o, void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!q || !k || !v || !idx || !o || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) ||
+        !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    return attend_impl(shape, g, q, k, v, idx, o, carve(g, workspace),
+                       static_cast<cudaStream_t>(stream));
+}
+
+bra_status bra_forward(const bra_shape* shape, const void* q, const void* k, const void* v,
+                       void* o, int32_t* idx, void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!q || !k || !v || !idx || !o || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) ||
+        !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    const Workspace w = carve(g, workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = route_impl(shape, g, q, k, idx, w, st);
+    if (rc != BRA_OK) return rc;
+    return attend_impl(shape, g, q, k, v, idx, o, w, st);
+}
+
+bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!workspace || !aligned16(workspace)) return BRA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* status = carve(g, workspace).status;
+    int host = 0;
+    if (cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BRA_ERR_CUDA;
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return BRA_ERR_CUDA;
+    if (host == kDevTimeout) return BRA_ERR_TIMEOUT;
+    if (host == kDevBadRoute) return BRA_ERR_BAD_ROUTE;
+    return host == 0 ? BRA_OK : BRA_ERR_CUDA;
+}
+
+const char* bra_status_string(bra_status status) {
+    switch (status) {
+        case BRA_OK: return "ok";
+        case BRA_ERR_INVALID_ARG: return "invalid argument";
+        case BRA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case BRA_ERR_CUDA: return "CUDA error";
+        case BRA_ERR_TIMEOUT: return "device-side wait timed out";
+        case BRA_ERR_BAD_ROUTE: return "routing index out of range";
+    }
+    return "unknown status";
+}
+
+int bra_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,143 @@
+/*
+ * bra.h -- C ABI of the B200 (sm_100a) Bi-Level Routing Attention library.
+ *
+ * Bi-Level Routing Attention (BRA) is the attention of BiFormer ("BiFormer:
+ * Vision Transformer with Bi-Level Routing Attention", Zhu et al., CVPR
+ * 2023).  The blog page "BiFormer Reshapes Visual Attention with Bi-Level
+ * Routing", Part 2 section 2.2 "The Overall BRA Flow", defines the steps this
+ * library runs, starting from projected Q, K, V:
+ *
+ *   region partition  the H x W map is cut into S x S regions of
+ *                     n = (H/S)(W/S) tokens (step 1);
+ *   region routing    Q^r, K^r = per-region means of Q and K; the region
+ *                     affinity A^r = Q^r (K^r)^T; I^r = row-wise top-k of A^r
+ *                     (step 3);
+ *   token attention   every query token of region r attends, with a
+ *                     softmax, over the tokens of the k regions I^r[r] (step 4).
+ *
+ * Conventions shared by every entry point
+ *  - Q, K, V, O are dense channels-last [B, H, W, C] tensors in device
+ *    memory, all of the element type ``dtype``; head h owns channels
+ *    [h*d, (h+1)*d) with d = C / heads, and every head is routed and attended
+ *    on its own.
+ *  - Regions are numbered row-major over the S x S grid, tokens row-major
+ *    inside a region.
+ *  - I^r is int32 [B, heads, S*S, topk] in device memory; each row lists its
+ *    regions by (affinity descending, lower index first on ties).
+ *  - A^r is computed in fp32 from fp32 region means and is not scaled; the
+ *    attention logits are scaled by 1/sqrt(d); the softmax and both products
+ *    accumulate in fp32; a bf16 O is rounded to nearest-even from fp32.
+ *  - The local-context term of step 4 (a 5x5 depthwise convolution of V) is
+ *    not part of these calls.
+ *  - Every buffer is owned by the caller.  The library allocates no device or
+ *    host memory and keeps no per-call state; its only global state is a
+ *    per-device cache of the kernels' launch attributes.
+ *  - Every call is asynchronous on ``stream`` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Arguments are checked on the host first; an
+ *    invalid call returns an error and launches nothing.
+ *  - Supported sizes: H % S == 0, W % S == 0, C % heads == 0, 1 <= topk <=
+ *    S*S, S*S <= 256, d == 32, B >= 0 (B == 0 or an empty map is a no-op).
+ *    Pointers must be 16-byte aligned.  The S constraint is the pages'
+ *    own (blog Part 3: S is chosen as a divisor of the map size so that no
+ *    padding is needed); d == 32 is the head size of every BiFormer stage.
+ *  - Thread safety: calls on different streams may run concurrently as long
+ *    as they do not share ``workspace`` or output buffers.
+ */
+#ifndef BRA_H
+#define BRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BRA_OK = 0,
+    BRA_ERR_INVALID_ARG = 1, /* sizes or pointers break the rules above     */
+    BRA_ERR_UNSUPPORTED = 2, /* valid BRA problem this build does not cover */
+    BRA_ERR_CUDA = 3,        /* a CUDA call or a kernel launch failed       */
+    BRA_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out          */
+    BRA_ERR_BAD_ROUTE = 5    /* bra_attend saw a routing index outside [0, S*S) */
+} bra_status;
+
+typedef enum { BRA_DTYPE_F32 = 0, BRA_DTYPE_BF16 = 1 } bra_dtype;
+
+/* One problem: feature map [B, H, W, C], heads, S x S regions, topk routes. */
+typedef struct {
+    int B, H, W, C;
+    int heads;
+    int S;
+    int topk;
+    int dtype; /* a bra_dtype */
+} bra_shape;
+
+/*
+ * Bytes of device workspace the calls below need for ``shape``: the fp32
+ * region means Q^r and K^r ([B, heads, S*S, d] each) followed by a 256-byte
+ * status block.  Returns 0 when ``shape`` is invalid.  The status block must
+ * hold zeros before the first call (zero the whole workspace once after
+ * allocating it); kernels only ever set it and bra_device_status clears it.
+ * The rest needs no initialisation.  The workspace may be reused by calls
+ * that are ordered on the GPU (e.g. one stream).
+ */
+size_t bra_workspace_bytes(const bra_shape* shape);
+
+/*
+ * Region-level routing (blog section 2.2 step 3): pools Q and K per region
+ * into the workspace, forms A^r = Q^r (K^r)^T per (batch, head) in fp32 and
+ * writes I^r = row-wise top-k to ``idx`` [B, heads, S*S, topk].
+ *   q, k       device, [B, H, W, C] of ``shape->dtype``, read only
+ *   idx        device int32 [B, heads, S*S, topk], written
+ *   workspace  device, bra_workspace_bytes(shape) bytes, scratch
+ * Errors: BRA_ERR_INVALID_ARG (bad sizes, NULL or misaligned pointer),
+ * BRA_ERR_UNSUPPORTED (d != 32, S*S > 256), BRA_ERR_CUDA (launch failed).
+ */
+bra_status bra_route(const bra_shape* shape, const void* q, const void* k, int32_t* idx,
+                     void* workspace, void* stream);
+
+/*
+ * Token-to-token attention over the routed regions (blog section 2.2 step 4):
+ * for every query token t of region r and head h,
+ *   O[t] = sum_j softmax_j(<q_t, k_j> / sqrt(d)) v_j
+ * where j runs over the tokens of the regions idx[b, h, r, 0..topk-1].  The
+ * routed K/V tiles are staged in shared memory and never written to HBM.
+ *   q, k, v    device, [B, H, W, C] of ``shape->dtype``, read only
+ *   idx        device int32 [B, heads, S*S, topk], read only; any routing
+ *              (it need not come from bra_route); an entry outside [0, S*S)
+ *              makes the kernel skip that region's outputs and record
+ *              BRA_ERR_BAD_ROUTE in the workspace status block
+ *   o          device, [B, H, W, C] of ``shape->dtype``, written
+ *   workspace  as for bra_route (only its status block is used)
+ * Errors: as bra_route.  Device-side problems are reported by
+ * bra_device_status.
+ */
+bra_status bra_attend(const bra_shape* shape, const void* q, const void* k, const void* v,
+                      const int32_t* idx, void* o, void* workspace, void* stream);
+
+/*
+ * The whole path: bra_route then bra_attend on the same stream, writing both
+ * the routing ``idx`` and the output ``o``.  Arguments as above.
+ */
+bra_status bra_forward(const bra_shape* shape, const void* q, const void* k, const void* v,
+                       void* o, int32_t* idx, void* workspace, void* stream);
+
+/*
+ * Reads (synchronising ``stream``) and clears the device status block in
+ * ``workspace``: BRA_OK, BRA_ERR_TIMEOUT (a bounded wait in a kernel gave up;
+ * that kernel's outputs are incomplete) or BRA_ERR_BAD_ROUTE.
+ */
+bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stream);
+
+/* Static English text for a status code. */
+const char* bra_status_string(bra_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int bra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BRA_H */

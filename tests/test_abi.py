@@ -1,0 +1,111 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every entry point
+that include/bra.h declares, and rejects bad arguments on the host before
+any CUDA call (no kernel is launched by these tests)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dynamic_sparse_attention_bra_b200 as bra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = []
+    for path in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(bra_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("bra_route", "bra_attend", "bra_forward", "bra_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(bra.library_path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(bra.EXPORTED_SYMBOLS) <= set(declared_functions())
+
+
+def test_version_and_strings():
+    assert bra._lib.bra_version() >= 100
+    assert bra.bra_status_string(0) == "ok"
+    assert "range" in bra.bra_status_string(5)
+
+
+S1 = dict(B=64, H=56, W=56, C=64, heads=2, S=7, topk=1, dtype="bf16")
+
+
+def shp(**kw):
+    a = dict(S1)
+    a.update(kw)
+    return bra.shape_for(a["B"], a["H"], a["W"], a["C"], a["heads"], a["S"], a["topk"], a["dtype"])
+
+
+def test_workspace_bytes():
+    s = shp()
+    means = 64 * 2 * 49 * 32 * 4
+    means = (means + 255) // 256 * 256
+    assert bra.bra_workspace_bytes(s) == 2 * means + 256
+    assert bra.bra_workspace_bytes(shp(B=0)) == 256
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(S=5), bra.BRA_ERR_INVALID_ARG),        # S does not divide 56
+    (dict(H=57), bra.BRA_ERR_INVALID_ARG),
+    (dict(topk=0), bra.BRA_ERR_INVALID_ARG),
+    (dict(topk=50), bra.BRA_ERR_INVALID_ARG),
+    (dict(heads=3), bra.BRA_ERR_INVALID_ARG),     # C % heads
+    (dict(B=-1), bra.BRA_ERR_INVALID_ARG),
+    (dict(C=0), bra.BRA_ERR_INVALID_ARG),
+    (dict(heads=1), bra.BRA_ERR_UNSUPPORTED),     # d = 64
+    (dict(C=128, heads=8), bra.BRA_ERR_UNSUPPORTED),  # d = 16
+    (dict(H=64, W=64, S=32, topk=1), bra.BRA_ERR_UNSUPPORTED),  # 1024 regions
+])
+def test_bad_shapes_rejected_before_launch(bad, code):
+    s = shp(**bad)
+    p = 1 << 20  # never dereferenced: the shape check fails first
+    assert bra._lib.bra_forward(ctypes.byref(s), p, p, p, p, p, p, None) == code
+    assert bra._lib.bra_route(ctypes.byref(s), p, p, p, p, None) == code
+    assert bra._lib.bra_attend(ctypes.byref(s), p, p, p, p, p, p, None) == code
+    assert bra.bra_workspace_bytes(s) == 0
+
+
+def test_bad_dtype_and_null_shape():
+    s = shp()
+    s.dtype = 7
+    assert bra._lib.bra_forward(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None) == bra.BRA_ERR_INVALID_ARG
+    assert bra._lib.bra_forward(None, 16, 16, 16, 16, 16, 16, None) == bra.BRA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(6))
+def test_null_and_misaligned_pointers(which):
+    s = shp()
+    good = [1 << 20] * 6
+    for bad in (0, (1 << 20) + 8):
+        ptrs = list(good)
+        ptrs[which] = bad
+        q, k, v, o, idx, ws = ptrs
+        assert bra._lib.bra_forward(ctypes.byref(s), q, k, v, o, idx, ws, None) == bra.BRA_ERR_INVALID_ARG
+        assert bra._lib.bra_attend(ctypes.byref(s), q, k, v, idx, o, ws, None) == bra.BRA_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The binding has no fallback: a missing library is an ImportError."""
+    import importlib.util
+    src = os.path.join(os.path.dirname(bra.__file__), "__init__.py")
+    pkg = tmp_path / "fakepkg"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(open(src).read())
+    spec = importlib.util.spec_from_file_location("fakepkg", pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,134 @@
+"""CUDA path vs the float64 oracle on the same seeded inputs, through the C ABI.
+
+Routing is compared under the rule in ``parity.py`` (bit-exact wherever the
+k-th/(k+1)-th affinity gap exceeds 1e-4 relative); O is compared with the
+oracle's token attention on the GPU's routing, max-abs within 1e-4 (fp32)
+or 2e-2 (bf16).  The five workload shapes run at full size, in the same
+launch configuration the benchmark times; the extra shapes cover ragged
+tiles, non-square regions, dense routing, a single region and the limits.
+"""
+import numpy as np
+import pytest
+
+import bra_inputs as bi
+import oracle
+from gpu_helpers import device_inputs, run_forward
+from parity import TOL, compare_routes
+
+pytestmark = pytest.mark.gpu
+
+
+def check_case(shape: bi.BraShape, seed: int, max_ambiguous_frac: float = 0.01):
+    inp = bi.make_inputs(shape, seed)
+    o_gpu, idx_gpu = run_forward(inp)
+    qr = oracle.region_pool(inp.q_f64, shape.heads, shape.S)
+    kr = oracle.region_pool(inp.k_f64, shape.heads, shape.S)
+    a = oracle.region_affinity(qr, kr)
+    rep = compare_routes(idx_gpu, a)
+    assert not rep.mismatches, f"{len(rep.mismatches)} routing rows differ, first {rep.mismatches[:3]}"
+    assert rep.ambiguous <= max(1, max_ambiguous_frac * rep.rows), rep.ambiguous
+    o_ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx_gpu, shape.heads, shape.S)
+    err = np.abs(o_gpu - o_ref).max()
+    assert err <= TOL[shape.dtype], f"max abs error {err:.3e} > {TOL[shape.dtype]}"
+    # the oracle's own routing gives the same O wherever the sets agree
+    return err, rep
+
+
+@pytest.mark.parametrize("name", list(bi.WORKLOADS))
+def test_workloads_full_size(name):
+    shape, seed = bi.WORKLOADS[name]
+    check_case(shape, seed)
+
+
+EXTRA = {
+    # name: (B, H, W, C, heads, S, topk, dtype)
+    "ragged_bf16": (2, 24, 24, 64, 2, 4, 3, "bf16"),        # n = 36: partial tiles
+    "ragged_f32": (2, 24, 24, 64, 2, 4, 3, "f32"),
+    "nonsquare_regions": (1, 18, 12, 32, 1, 6, 5, "bf16"),  # 3x2 tokens per region
+    "wide_map": (1, 16, 48, 64, 2, 4, 2, "bf16"),           # 4x12 tokens per region
+    "dense_topk": (1, 16, 16, 64, 2, 4, 16, "bf16"),        # k = S^2: full attention
+    "single_region": (2, 16, 20, 64, 2, 1, 1, "bf16"),      # n = 320: several query tiles
+    "single_token_regions": (2, 8, 8, 64, 2, 8, 4, "bf16"), # n = 1
+    "max_regions": (1, 32, 32, 32, 1, 16, 8, "bf16"),       # R = 256
+    "many_heads": (1, 14, 14, 512, 16, 7, 16, "bf16"),
+    "long_route_f32": (1, 32, 32, 32, 1, 4, 12, "f32"),     # 768 keys per query
+}
+
+
+@pytest.mark.parametrize("name", list(EXTRA))
+def test_extra_shapes(name):
+    B, H, W, C, heads, S, topk, dtype = EXTRA[name]
+    check_case(bi.BraShape(B, H, W, C, heads, S, topk, dtype), 100 + len(name))
+
+
+def test_repeatable_bitwise():
+    shape, seed = bi.WORKLOADS["stage2"]
+    inp = bi.make_inputs(shape, seed)
+    o1, i1 = run_forward(inp)
+    o2, i2 = run_forward(inp)
+    assert (i1 == i2).all() and (o1 == o2).all()
+
+
+def test_route_then_attend_equals_forward():
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape, seed = bi.WORKLOADS["stage3"]
+    inp = bi.make_inputs(shape, seed)
+    q, k, v = device_inputs(inp)
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device="cuda")
+    o = torch.empty_like(q)
+    bra.bra_route(s, q, k, idx, ws)
+    bra.bra_attend(s, q, k, v, idx, o, ws)
+    o2, idx2 = bra.forward(q, k, v, shape.heads, shape.S, shape.topk)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(o.view(torch.int16), o2.view(torch.int16))
+
+
+def test_attend_with_given_routing():
+    """bra_attend takes any routing, e.g. the oracle's own."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape = bi.BraShape(2, 16, 16, 64, 2, 4, 3, "bf16")
+    inp = bi.make_inputs(shape, 9)
+    _, idx_or = oracle.bra_forward(inp.q_f64, inp.k_f64, inp.v_f64, shape.heads, shape.S, shape.topk)
+    idx_or = np.ascontiguousarray(idx_or[..., ::-1])  # any order is a valid routing
+    q, k, v = device_inputs(inp)
+    s = bra.shape_for(*[getattr(shape, f) for f in "B H W C heads S topk".split()], shape.dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+    bra.bra_attend(s, q, k, v, torch.from_numpy(idx_or).cuda(), o, ws)
+    assert bra.bra_device_status(s, ws) == bra.BRA_OK
+    o_ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx_or, shape.heads, shape.S)
+    assert np.abs(o.float().cpu().numpy() - o_ref).max() <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("bad_value", [-1, 16, 1 << 30])
+def test_bad_route_is_reported_not_read(bad_value):
+    """An out-of-range routing index is caught by the kernel's own check: the
+    region is skipped and the status block says BRA_ERR_BAD_ROUTE."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape = bi.BraShape(1, 16, 16, 64, 2, 4, 2, "bf16")
+    inp = bi.make_inputs(shape, 3)
+    q, k, v = device_inputs(inp)
+    s = bra.shape_for(1, 16, 16, 64, 2, 4, 2, "bf16")
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    idx = torch.zeros((1, 2, 16, 2), dtype=torch.int32, device="cuda")
+    idx[0, 1, 5, 1] = bad_value
+    o = torch.zeros_like(q)
+    bra.bra_attend(s, q, k, v, idx, o, ws)
+    assert bra.bra_device_status(s, ws) == bra.BRA_ERR_BAD_ROUTE
+    assert bra.bra_device_status(s, ws) == bra.BRA_OK  # cleared by the read
+
+
+def test_empty_batch_is_a_noop():
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    s = bra.shape_for(0, 56, 56, 64, 2, 7, 1, "bf16")
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    buf = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros(4, dtype=torch.int32, device="cuda")
+    bra.bra_forward(s, buf, buf, buf, buf, idx, ws)
+    assert bra.bra_device_status(s, ws) == bra.BRA_OK
