@@ -25,6 +25,7 @@ import os
 __all__ = [
     "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
     "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
+    "bra_route_noalloc",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -35,7 +36,8 @@ BRA_OK, BRA_ERR_INVALID_ARG, BRA_ERR_UNSUPPORTED, BRA_ERR_CUDA, BRA_ERR_TIMEOUT,
 BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
-                    "bra_device_status", "bra_status_string", "bra_version")
+                    "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc")
+NOALLOC_MAX_MEANS = 1 << 20  # BRA_NOALLOC_MAX_MEANS
 
 
 class BraShape(ctypes.Structure):
@@ -63,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.bra_attend.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_device_status.argtypes = [sp, vp, vp]
+    lib.bra_route_noalloc.argtypes = [sp, vp, vp, vp, vp]
+    lib.bra_route_noalloc.restype = ctypes.c_int
     for f in (lib.bra_route, lib.bra_attend, lib.bra_forward, lib.bra_device_status):
         f.restype = ctypes.c_int
     lib.bra_status_string.argtypes = [ctypes.c_int]
@@ -119,6 +123,14 @@ def bra_attend(shape: BraShape, q, k, v, idx, o, workspace, stream=None) -> None
 def bra_forward(shape: BraShape, q, k, v, o, idx, workspace, stream=None) -> None:
     _check(_lib.bra_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(idx),
                             _ptr(workspace), _stream(stream)), "bra_forward")
+
+
+def bra_route_noalloc(shape: BraShape, q, k, idx, stream=None) -> None:
+    """bra_route with the library's own fixed scratch: for callers that cannot
+    allocate device memory (see include/bra.h for the size limit and the
+    rule that overlapping calls race)."""
+    _check(_lib.bra_route_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(idx), _stream(stream)),
+           "bra_route_noalloc")
 
 
 def bra_device_status(shape: BraShape, workspace, stream=None) -> int:

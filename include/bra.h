@@ -130,6 +130,27 @@ bra_status bra_forward(const bra_shape* shape, const void* q, const void* k, con
  */
 bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stream);
 
+/*
+ * Routing without a caller-supplied workspace.  The pages describe nothing
+ * like it: it exists for callers that cannot allocate device memory, such as
+ * plugins inside a host framework that owns all device memory and hands out
+ * none, or loops that must not call cudaMalloc because it can synchronise
+ * the whole device.  It writes the same ``idx`` as bra_route.
+ *
+ * The scratch for Q^r and K^r is a fixed array inside the library (every
+ * GPU that loads the library holds it, 2 * BRA_NOALLOC_MAX_MEANS floats =
+ * 8 MiB, until the process exits).  Limit: B * heads * S*S * d must not
+ * exceed BRA_NOALLOC_MAX_MEANS, else BRA_ERR_UNSUPPORTED (and nothing is
+ * launched); other argument errors are those of bra_route.  The first call
+ * on a device looks up the array's device address there (the caller's
+ * current device); make that first call before any stream capture.  All
+ * calls share the array, so calls that overlap on the GPU race: order them
+ * (e.g. one stream).  Allocates nothing, host or device.
+ */
+#define BRA_NOALLOC_MAX_MEANS (1u << 20)
+bra_status bra_route_noalloc(const bra_shape* shape, const void* q, const void* k, int32_t* idx,
+                             void* stream);
+
 /* Static English text for a status code. */
 const char* bra_status_string(bra_status status);
 
