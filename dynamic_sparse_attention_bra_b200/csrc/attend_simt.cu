@@ -25,18 +25,30 @@ bra_attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     __shared__ __align__(16) float ks[kSimtKeyBlock][LD];
     __shared__ __align__(16) float vs[kSimtKeyBlock][LD];
     __shared__ int routes[kMaxRegions];
-    __shared__ int bad;
+    __shared__ uint32_t seen[kMaxRegions / 32];
+    __shared__ int bad, nroutes;
 
     const int chunk_id = blockIdx.x % plan.chunks, r = blockIdx.x / plan.chunks;
     const int h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x;
     const int32_t* row = idx + (((size_t)b * g.heads + h) * g.R + r) * g.topk;
-    if (tid == 0) bad = 0;
-    __syncthreads();
-    for (int m = tid; m < g.topk; m += kSimtThreads) {
-        const int rr = row[m];
-        if (rr < 0 || rr >= g.R) bad = 1;
-        routes[m] = rr;
+    // The routed regions, each once: a caller-given row may repeat a region,
+    // and attention runs over the union of the routed regions' tokens.
+    if (tid == 0) {
+        bad = 0;
+        nroutes = 0;
+        for (int w = 0; w < kMaxRegions / 32; ++w) seen[w] = 0;
+        for (int m = 0; m < g.topk; ++m) {
+            const int rr = row[m];
+            if (rr < 0 || rr >= g.R) {
+                bad = 1;
+                break;
+            }
+            if (!((seen[rr >> 5] >> (rr & 31)) & 1u)) {
+                seen[rr >> 5] |= 1u << (rr & 31);
+                routes[nroutes++] = rr;
+            }
+        }
     }
     __syncthreads();
     if (bad) {
@@ -65,7 +77,7 @@ bra_attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
 #pragma unroll
     for (int c = 0; c < D; ++c) acc[c] = 0.f;
 
-    const int kn = g.topk * g.n;
+    const int kn = nroutes * g.n;
     for (int j0 = 0; j0 < kn; j0 += kSimtKeyBlock) {
         const int nb = min(kSimtKeyBlock, kn - j0);
         __syncthreads();

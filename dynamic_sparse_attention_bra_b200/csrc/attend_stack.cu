@@ -1,0 +1,583 @@
+// Persistent, warp-specialised tcgen05 attention for regions of 16..64 tokens
+// (blog "BiFormer Reshapes Visual Attention with Bi-Level Routing", Part 2
+// section 2.2, step 4: gather the routed key-value regions, then token
+// attention over them).
+//
+// Tiling.  A tile is 128 query rows of one (batch, head) split into two
+// 64-row halves; a half holds Gq whole query regions (Gq * n <= 64).  Each
+// query region r brings its own key list: the tokens of its routed regions
+// I^r[r][0..topk), kn = topk * n keys, stacked slot after slot, so half h
+// multiplies Q_h [64 x 32] by K_h^T [32 x Gq*kn] with one M = 64 tcgen05.mma
+// per 16 channels.  The two halves' accumulators share TMEM columns: half 0
+// lands in lanes 0-15 of each 32-lane quadrant, half 1 in lanes 16-31.  Row
+// m of a half belongs to slot m / n, so its valid scores are exactly the
+// window [slot * kn, slot * kn + kn) of its TMEM row -- one 16-row group
+// never straddles two slots because n is a multiple of 16, which makes the
+// window the same for all lanes of a warp.  No score outside a window is
+// ever read, and P is zero outside the windows (each P row only ever writes
+// its own window), so O_h = P_h V_h (M = 64, N = 32) needs no masking either.
+//
+// Roles (192 threads, one CTA per SM, tiles strided by the grid):
+//   warp 0     producer: reads the tile's routes, issues TMA box loads of the
+//              query regions and of every routed key/value region straight
+//              from the [B, H, W, C] maps into a ring of shared-memory stages
+//              (64-byte swizzle), completion counted on the stage's mbarrier;
+//   warp 1     one lane issues the MMAs: S = Q K^T for tile i + 1 (double
+//              buffered in TMEM) before P V for tile i;
+//   warps 2-5  softmax and epilogue, one query row per thread: read the row's
+//              window of S, base-2 softmax in fp32, P as bf16 into 128-byte
+//              swizzled shared memory, then O = (P V) / l to global memory.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// kDevTimeout, stops all roles, drains its MMAs and frees TMEM.
+#include <cuda.h>
+
+#include "attend_tc.h"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+#include "tma_host.h"
+
+namespace bra {
+namespace {
+
+constexpr int kMaxSlots = 4;    // 64 rows / 16 tokens
+constexpr int kMaxRoutes = 16;  // kn <= 256 with n >= 16
+constexpr int kMaxStages = 8;
+constexpr int kMaxSBuf = 8;
+constexpr uint32_t kWait = 1u << 22;
+constexpr uint32_t kSpinLimit = 1u << 26;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kSmemBudget = 227 * 1024;
+
+struct StackPlan {
+    int Gq;                 // query regions per half
+    int kn;                 // keys per query region
+    int N;                  // keys per half = Gq * kn (MMA N of Q K^T)
+    int halves;             // half tiles per (batch, head)
+    int tiles_bh;           // tiles per (batch, head)
+    int tiles;              // all tiles
+    int stages;             // shared-memory ring depth
+    int nsb;                // S buffers in TMEM
+    int np;                 // P buffers in shared memory
+    int items;              // (slot, route) pairs of a tile: 2 * Gq * topk <= 32
+    int wgs;                // softmax warp groups (1 or 2)
+    int pdepth;             // P buffers per warp group (2: a tile's epilogue waits one tile)
+    uint32_t stage_bytes;   // Q (2 x 64 rows) + K + V of one tile
+    uint32_t k_off, v_off;  // offsets inside a stage
+    uint32_t p_half;        // one half of a P buffer: ceil(N / 64) atoms of 64 rows x 128 B
+    uint32_t p_off;         // offset of the P buffers
+    uint32_t ones_off;      // offset of a bf16 ones tile [16][N] (row sums of P by MMA)
+    uint32_t bar_off;       // offset of barriers and tile metadata
+    uint32_t smem_bytes;    // dynamic shared memory requested (incl. alignment slack)
+    uint32_t tmem_cols;     // nsb S buffers of N columns, rounded up to a power of two
+};
+
+struct TileMeta {
+    int b, h;
+    int reg[2][kMaxSlots];         // query region of each slot, -1 if none
+    uint32_t live[2][kMaxSlots];   // bit m: route m loaded (in range, first occurrence)
+};
+
+struct Barriers {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t s_full[kMaxSBuf], o_full[kMaxSBuf], s_free[kMaxSBuf];
+    uint64_t p_full[4];
+    uint64_t drain[2];
+    TileMeta meta[kMaxStages];
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ bool aborted(Barriers* sb) {
+    return *reinterpret_cast<volatile int*>(&sb->abort) != 0;
+}
+
+__device__ __forceinline__ void set_abort(Barriers* sb, int* status) {
+    *reinterpret_cast<volatile int*>(&sb->abort) = 1;
+    raise_status(status, kDevTimeout);
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Barriers* sb,
+                                              int* status) {
+    for (uint32_t i = 0; i < kWait; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023) == 1023 && aborted(sb)) return false;
+    }
+    set_abort(sb, status);
+    return false;
+}
+
+// Per-row state kept from a tile's softmax until its epilogue.
+struct RowState {
+    int region, b, h;
+    float l;
+};
+
+constexpr int kProd = 2;   // producer warps (tiles alternate between them)
+constexpr int kCtrl = kProd + 2;  // + the S issuer warp and the P V issuer warp
+
+// WGS softmax warp groups (1 or 2); KN64: every window is exactly 64 keys.
+template <int WGS, bool KN64>
+__global__ void __launch_bounds__(32 * kCtrl + 128 * WGS, 1)
+bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                        const __grid_constant__ CUtensorMap tv, const int32_t* __restrict__ idx,
+                        __nv_bfloat16* __restrict__ o, Geometry g, StackPlan p, int* status) {
+    constexpr int kThreads = 32 * kCtrl + 128 * WGS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_addr(smem);
+    Barriers* sb = reinterpret_cast<Barriers*>(smem + p.bar_off);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int my_tiles =
+        (int)blockIdx.x < p.tiles ? (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            ptx::mbar_init(&sb->full[s], 1);
+            ptx::mbar_init(&sb->empty[s], 1);
+        }
+        for (int b = 0; b < p.nsb; ++b) {
+            ptx::mbar_init(&sb->s_full[b], 1);
+            ptx::mbar_init(&sb->o_full[b], 1);
+            ptx::mbar_init(&sb->s_free[b], 128);
+        }
+        for (int b = 0; b < p.np; ++b) ptx::mbar_init(&sb->p_full[b], 128);
+        ptx::mbar_init(&sb->drain[0], 1);
+        ptx::mbar_init(&sb->drain[1], 1);
+        sb->abort = 0;
+        ptx::mbar_init_fence();
+    }
+    if (warp == kProd) {
+        ptx::tmem_alloc(&sb->tmem, p.tmem_cols);
+        ptx::tmem_relinquish();
+        ptx::tc_fence_before();
+    }
+    // Zero every operand buffer once: stale rows outside a tile's loaded boxes
+    // are then always finite, and P stays zero outside each row's window.
+    for (uint32_t i = threadIdx.x; i < p.ones_off / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+    // A tile of bf16 ones (same shape as one V half): P times it gives every
+    // row's sum of P on the tensor core.
+    for (uint32_t i = p.ones_off / 16 + threadIdx.x; i < p.bar_off / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sb->tmem;
+    // Everything above overlaps the routing kernel; from here on the routes
+    // are read and O is written.
+    grid_dependency_wait();
+
+    if (warp < kProd) {
+        // ------------------------------------------------------------ producer
+        // Producer warp w loads tiles w, w + kProd, ...  Lane j first owns item
+        // j = (half, slot, route m) of the tile (reads its route, checks it),
+        // then the tile's boxes -- one query box per slot, one key and one value
+        // box per live item -- go out one box per lane in a single TMA
+        // instruction (copies from one thread are processed in order, copies
+        // from different lanes in parallel), rotated across tiles so that
+        // successive tiles use different lanes.  Routes of the warp's next tile
+        // are read while this tile's copies are issued.
+        if (lane == 0 && warp == 0) {
+            ptx::tma_prefetch_desc(&tq);
+            ptx::tma_prefetch_desc(&tk);
+            ptx::tma_prefetch_desc(&tv);
+        }
+        const bool item = lane < p.items;
+        const int per_half = p.Gq * g.topk;
+        const int half = item ? lane / per_half : 0;
+        const int slot = item ? (lane / g.topk) % p.Gq : 0;
+        const int m = item ? lane % g.topk : 0;
+        const int lane0 = lane - m;  // lane of route 0 of this slot
+        const uint32_t slot_lanes = (g.topk >= 32 ? 0xffffffffu : ((1u << g.topk) - 1u)) << lane0;
+        const uint32_t nbytes_region = (uint32_t)g.n * 64u;
+        const int nq = 2 * p.Gq;                 // query boxes of a tile
+        const int nboxes = nq + 2 * p.items;     // + key and value boxes
+        auto fetch = [&](int i, int& reg) -> int {
+            const int t = blockIdx.x + i * gridDim.x;
+            const int bh = t / p.tiles_bh, tt = t - bh * p.tiles_bh;
+            const int ht = tt * 2 + half;
+            const int r = ht * p.Gq + slot;
+            reg = (item && ht < p.halves && r < g.R) ? r : -1;
+            return reg >= 0 ? __ldg(idx + ((size_t)bh * g.R + r) * g.topk + m) : 0;
+        };
+        int cur_reg = -1, nxt_reg = -1;
+        int cur = warp < my_tiles ? fetch(warp, cur_reg) : 0;
+        for (int i = warp; i < my_tiles; i += kProd) {
+            const int nxt = i + kProd < my_tiles ? fetch(i + kProd, nxt_reg) : 0;
+            const int s = i % p.stages;
+            if (i >= p.stages && !wait_or_abort(&sb->empty[s], ((i / p.stages) - 1) & 1, sb, status))
+                break;
+            const int t = blockIdx.x + i * gridDim.x;
+            const int bh = t / p.tiles_bh;
+            const int b = bh / g.heads, hd = bh - b * g.heads;
+            const bool valid = cur_reg >= 0;
+            const uint32_t bad = __ballot_sync(0xffffffffu, valid && (cur < 0 || cur >= g.R));
+            const bool slot_ok = valid && !(bad & slot_lanes);
+            if (valid && !slot_ok && m == 0) raise_status(status, kDevBadRoute);
+            bool dup = false;
+            for (int dd = 1; dd < g.topk; ++dd) {
+                const int other = __shfl_up_sync(0xffffffffu, cur, dd);
+                if (dd <= m && other == cur) dup = true;
+            }
+            const bool live = slot_ok && !dup;
+            const uint32_t live_lanes = __ballot_sync(0xffffffffu, live);
+            const uint32_t ok_lanes = __ballot_sync(0xffffffffu, slot_ok && m == 0);
+            TileMeta& M = sb->meta[s];
+            if (item && m == 0) {
+                M.reg[half][slot] = slot_ok ? cur_reg : -1;
+                M.live[half][slot] = (live_lanes & slot_lanes) >> lane0;
+            }
+            if (lane == 0) {
+                M.b = b;
+                M.h = hd;
+            }
+            const uint32_t bytes = (uint32_t)(__popc(ok_lanes) + 2 * __popc(live_lanes)) * nbytes_region;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&sb->full[s], bytes);
+            __syncwarp();
+            const uint32_t stage = sbase + (uint32_t)s * p.stage_bytes;
+            const int rot = (i / kProd * nboxes) & 31;
+            for (int j0 = 0; j0 < nboxes; j0 += 32) {
+                const int j = j0 + ((lane - rot) & 31);  // box this lane issues
+                // the item behind box j: query box j -> slot lane (j * topk), K/V box -> item
+                const int it = j < nq ? j * g.topk : (j - nq) >> 1;
+                const int src = it < 32 ? it : 0;
+                const int x_cur = __shfl_sync(0xffffffffu, cur, src);
+                const int x_reg = __shfl_sync(0xffffffffu, cur_reg, src);
+                if (j >= nboxes) continue;
+                const int x_half = it / per_half, x_slot = (it / g.topk) % p.Gq, x_m = it % g.topk;
+                if (j < nq) {
+                    if ((ok_lanes >> it) & 1u) {
+                        const int ri = x_reg / g.S, rj = x_reg - ri * g.S;
+                        ptx::tma_load_4d(stage + x_half * 4096 + x_slot * nbytes_region, &tq, hd * 32, rj * g.ws,
+                                         ri * g.hs, b, &sb->full[s]);
+                    }
+                } else if ((live_lanes >> it) & 1u) {
+                    const int qi = x_cur / g.S, qj = x_cur - qi * g.S;
+                    const uint32_t koff = (uint32_t)(x_half * p.N + x_slot * p.kn + x_m * g.n) * 64u;
+                    const bool is_v = (j - nq) & 1;
+                    ptx::tma_load_4d(stage + (is_v ? p.v_off : p.k_off) + koff, is_v ? (const void*)&tv : (const void*)&tk,
+                                     hd * 32, qj * g.ws, qi * g.hs, b, &sb->full[s]);
+                }
+            }
+            cur = nxt;
+            cur_reg = nxt_reg;
+        }
+    } else if (warp == kProd) {
+        // ------------------------------------------------------- S = Q K^T issuer
+        // One lane issues S for every tile in order as soon as the tile's stage
+        // is loaded and its TMEM buffer is released; it never waits on P.
+        if (lane == 0) {
+            const uint32_t idesc_qk = ptx::idesc_bf16_f32(64, p.N, false, false);
+            for (int i = 0; i < my_tiles; ++i) {
+                const int s = i % p.stages, sbuf = i % p.nsb;
+                if (!wait_or_abort(&sb->full[s], (i / p.stages) & 1, sb, status)) break;
+                if (i >= p.nsb && !wait_or_abort(&sb->s_free[sbuf], ((i / p.nsb) - 1) & 1, sb, status)) break;
+                ptx::tc_fence_after();
+                const uint32_t stage = sbase + (uint32_t)s * p.stage_bytes;
+                // halves alternate so that consecutive MMAs accumulate into different tiles
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint64_t a = ptx::smem_desc(stage + half * 4096 + kk * 32, 16, 512, ptx::kSwizzle64B);
+                        const uint64_t bd = ptx::smem_desc(stage + p.k_off + (uint32_t)half * p.N * 64 + kk * 32, 16,
+                                                           512, ptx::kSwizzle64B);
+                        ptx::mma_bf16(tmem + sbuf * p.N + ((uint32_t)(half * 16) << 16), a, bd, idesc_qk, kk);
+                    }
+                }
+                ptx::mma_commit(&sb->s_full[sbuf]);
+            }
+            // Let every MMA this thread issued finish before TMEM is freed.
+            ptx::mma_commit(&sb->drain[0]);
+            ptx::mbar_wait(&sb->drain[0], 0, kWait);
+        }
+        __syncwarp();
+    } else if (warp == kProd + 1) {
+        // --------------------------------------------------- O = P V issuer
+        // One lane issues P V (and the row sums P x ones) for every tile in
+        // order as soon as its P is written, then releases the stage.
+        if (lane == 0) {
+            // N = 48: columns 0..31 are V, 32..47 come from a tile of ones, so the
+            // same MMA leaves the row sums of P next to O.
+            const uint32_t idesc_pv = ptx::idesc_bf16_f32(64, 48, false, true);
+            const uint32_t ones = sbase + p.ones_off;
+            for (int i = 0; i < my_tiles; ++i) {
+                const int s = i % p.stages, sbuf = i % p.nsb, pb = i % p.np;
+                if (!wait_or_abort(&sb->p_full[pb], (i / p.np) & 1, sb, status)) break;
+                ptx::tc_fence_after();
+                const uint32_t stage = sbase + (uint32_t)s * p.stage_bytes;
+                const uint32_t pbase = sbase + p.p_off + (uint32_t)pb * 2u * p.p_half;
+                for (int kk = 0; kk < p.N / 16; ++kk) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t d = tmem + sbuf * p.N + ((uint32_t)(half * 16) << 16);
+                        const uint64_t a = ptx::smem_desc(pbase + half * p.p_half + (kk >> 2) * 8192 + (kk & 3) * 32,
+                                                          16, 1024, ptx::kSwizzle128B);
+                        // B: V rows (N 0..31) and, one leading-byte offset further, the ones (N 32..63)
+                        const uint32_t vaddr = stage + p.v_off + (uint32_t)half * p.N * 64 + kk * 1024;
+                        const uint64_t bd = ptx::smem_desc(vaddr, ones + kk * 1024 - vaddr, 512, ptx::kSwizzle64B);
+                        ptx::mma_bf16(d, a, bd, idesc_pv, kk);
+                    }
+                }
+                ptx::mma_commit(&sb->o_full[sbuf]);
+                ptx::mma_commit(&sb->empty[s]);
+            }
+            ptx::mma_commit(&sb->drain[1]);
+            ptx::mbar_wait(&sb->drain[1], 0, kWait);
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------- softmax + epilogue
+        // Warp group wg owns tiles wg, wg + WGS, ...; with two groups one
+        // group's P V and epilogue overlap the other group's softmax.
+        const int wg = (warp - kCtrl) >> 2;
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int half = lane >> 4;
+        const int m = 16 * q + (lane & 15);  // row within the half
+        const int slot = m / g.n;            // same for the whole warp
+        const int tok = m - slot * g.n;
+        const bool slot_ok = slot < p.Gq;
+        const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+        const uint32_t full_live = g.topk >= 32 ? 0xffffffffu : ((1u << g.topk) - 1u);
+        const float sl = kLog2e * rsqrtf(32.f);
+
+        // O = (P V) / l for tile j, then release its TMEM buffer.
+        auto epilogue = [&](int j, const RowState& st) -> bool {
+            const int sbuf = j % p.nsb;
+            if (!wait_or_abort(&sb->o_full[sbuf], (j / p.nsb) & 1, sb, status)) return false;
+            ptx::tc_fence_after();
+            uint32_t r[32], rl[16];
+            float l = 0.f;
+            if (slot_ok) {
+                ptx::tmem_ld32(tmem + lane_addr + sbuf * p.N, r);
+                ptx::tmem_ld16(tmem + lane_addr + sbuf * p.N + 32, rl);
+                ptx::tmem_ld_wait();
+                l = __uint_as_float(rl[0]);
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&sb->s_free[sbuf]);
+            if (st.region >= 0 && l > 0.f) {
+                const float inv = 1.f / l;
+                int4* dst = reinterpret_cast<int4*>(o + token_offset(g, st.b, st.region, tok) + (size_t)st.h * 32);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[8 * c + 2 * e]) * inv,
+                                                                        __uint_as_float(r[8 * c + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+                    }
+                    __stcs(dst + c, make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]));  // streamed: O is not re-read
+                }
+            }
+            return true;
+        };
+
+        RowState prev = {-1, 0, 0, 0.f};
+        bool ok = true;
+        int last = -1;
+        for (int i = wg; ok && i < my_tiles; i += WGS) {
+            const int s = i % p.stages, sbuf = i % p.nsb, pb = i % p.np;
+            if (!wait_or_abort(&sb->full[s], (i / p.stages) & 1, sb, status)) break;
+            if (!wait_or_abort(&sb->s_full[sbuf], (i / p.nsb) & 1, sb, status)) break;
+            ptx::tc_fence_after();
+            const TileMeta& M = sb->meta[s];
+            RowState cur;
+            cur.region = slot_ok ? M.reg[half][slot] : -1;
+            cur.b = M.b;
+            cur.h = M.h;
+            const uint32_t live = slot_ok ? M.live[half][slot] : 0u;
+            const bool all_live = live == full_live;
+            float l = 0.f;
+            if (slot_ok) {
+                const uint32_t col0 = sbuf * p.N + slot * p.kn;
+                const uint32_t prow = sbase + p.p_off + (uint32_t)pb * 2u * p.p_half + half * p.p_half + m * 128;
+                // segment j (16 columns) of the window belongs to route j * 16 / n
+                auto seg_mask = [&](int c) -> uint32_t {
+                    if (all_live) return 0xffffffffu;
+                    const int r0 = (c >> 4) * 16 / g.n, r1 = ((c >> 4) + 1) * 16 / g.n;
+                    return (((live >> r0) & 1u) ? 0x0000ffffu : 0u) | (((live >> r1) & 1u) ? 0xffff0000u : 0u);
+                };
+                auto write_p = [&](int c, const uint32_t* packed) {
+                    const int col = slot * p.kn + c;  // window column inside the half's P
+                    const uint32_t atom = prow + (uint32_t)(col >> 6) * 8192u;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const int chunk = ((col & 63) >> 3) + cc;
+                        ptx::st_shared_v4(atom + ((chunk ^ (m & 7)) << 4), packed[4 * cc], packed[4 * cc + 1],
+                                          packed[4 * cc + 2], packed[4 * cc + 3]);
+                    }
+                };
+                // p for 32 scores of chunk c (fp32 exponentials, rounded to bf16)
+                auto exp_chunk = [&](const uint32_t* r, uint32_t km, float msl, uint32_t* packed) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ((km >> (2 * e)) & 1u) ? ptx::ex2(fmaf(__uint_as_float(r[2 * e]), sl, -msl)) : 0.f;
+                        const float p1 = ((km >> (2 * e + 1)) & 1u) ? ptx::ex2(fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)) : 0.f;
+                        const __nv_bfloat162 pbf = __floats2bfloat162_rn(p0, p1);
+                        packed[e] = *reinterpret_cast<const uint32_t*>(&pbf);
+                    }
+                };
+                if (KN64 && __all_sync(0xffffffffu, all_live)) {
+                    // Every route of every row of this warp is live: no masks.
+                    // Two 32-column TMEM reads for the max, two more for p, so no
+                    // more than 32 scores are live in registers at a time.
+                    float m8[8];
+                    {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tmem + lane_addr + col0, r);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(r[e]);
+#pragma unroll
+                        for (int e = 8; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(r[e]));
+                        ptx::tmem_ld32(tmem + lane_addr + col0 + 32, r);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(r[e]));
+                    }
+                    const float msl = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                            fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl;
+                    // p = 2^(s * sl - max) on bf16 pairs: P enters the MMA as bf16
+                    // anyway, and the row sums come from the same bf16 values (P x ones).
+#pragma unroll
+                    for (int c = 0; c < 64; c += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_ld_wait();
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            packed[e] = ptx::ex2_bf16x2(ptx::pack_bf16x2(fmaf(__uint_as_float(r[2 * e]), sl, -msl),
+                                                                         fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)));
+                        write_p(c, packed);
+                    }
+                } else {
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    for (int c = 0; c < p.kn; c += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_ld_wait();
+                        const uint32_t km = seg_mask(c);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            m4[e & 3] = fmaxf(m4[e & 3], ((km >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY);
+                    }
+                    const float msl = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
+                    for (int c = 0; c < p.kn; c += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_ld_wait();
+                        uint32_t packed[16];
+                        exp_chunk(r, seg_mask(c), msl, packed);
+                        write_p(c, packed);
+                    }
+                }
+            }
+            cur.l = l;
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&sb->p_full[pb]);
+            if (p.pdepth == 2) {
+                // This group's previous tile finishes while this tile's P V runs.
+                if (last >= 0) ok = epilogue(last, prev);
+                prev = cur;
+                last = i;
+            } else {
+                ok = epilogue(i, cur);
+            }
+        }
+        if (ok && last >= 0) epilogue(last, prev);
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kProd) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+bool make_stack_plan(const Geometry& g, StackPlan* p) {
+    if (g.d != 32 || g.n % 16 != 0 || g.n > 64) return false;
+    const int kn = g.topk * g.n;
+    if (kn > 256 || kn % 32 != 0 || g.topk > kMaxRoutes) return false;
+    p->kn = kn;
+    p->Gq = 64 / g.n;
+    if (p->Gq * kn > 256) p->Gq = 256 / kn;
+    if (p->Gq > g.R) p->Gq = g.R;
+    if (p->Gq < 1) return false;
+    p->items = 2 * p->Gq * g.topk;
+    if (p->items > 32) return false;
+    p->N = p->Gq * kn;
+    if (p->N < 64) return false;  // the O block (32 columns) and its row sums (16) reuse S
+    p->halves = (g.R + p->Gq - 1) / p->Gq;
+    p->tiles_bh = (p->halves + 1) / 2;
+    const long long tiles = (long long)g.B * g.heads * p->tiles_bh;
+    if (tiles > 0x7fffffffLL) return false;
+    p->tiles = (int)tiles;
+    const uint32_t kv = (uint32_t)2 * p->N * 64;  // two halves of N rows of 64 B
+    p->k_off = 8192;
+    p->v_off = 8192 + kv;
+    p->stage_bytes = 8192 + 2 * kv;
+    p->p_half = (uint32_t)((p->N + 63) / 64) * 8192u;
+    const uint32_t misc = (uint32_t)((sizeof(Barriers) + 1023) / 1024 * 1024);
+    const uint32_t ones_bytes = (uint32_t)p->N * 64u;  // N keys x 64 B of bf16 ones
+    // Softmax warp groups x P buffers per group, most overlap first, as long
+    // as a load ring of at least 3 stages (2 for the last option) remains.
+    static const int kOptions[4][2] = {{2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    int stages = 0;
+    bool found = false;
+    for (int o = 0; o < 4 && !found; ++o) {
+        p->wgs = kOptions[o][0];
+        p->pdepth = kOptions[o][1];
+        p->np = p->wgs * p->pdepth;
+        const uint32_t used = 1024 + misc + ones_bytes + (uint32_t)p->np * 2u * p->p_half;
+        stages = used < kSmemBudget ? (int)((kSmemBudget - used) / p->stage_bytes) : 0;
+        found = stages >= (o == 3 ? 2 : 3);
+    }
+    if (!found) return false;
+    if (stages > kMaxStages) stages = kMaxStages;
+    p->stages = stages;
+    p->p_off = (uint32_t)stages * p->stage_bytes;
+    p->ones_off = p->p_off + (uint32_t)p->np * 2u * p->p_half;
+    p->bar_off = p->ones_off + ones_bytes;
+    p->smem_bytes = p->bar_off + (uint32_t)sizeof(Barriers) + 1024;
+    if (512 / p->N < 2) return false;
+    p->nsb = 512 / p->N >= kMaxSBuf ? kMaxSBuf : 512 / p->N;
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(p->nsb * p->N)) cols <<= 1;
+    p->tmem_cols = cols;
+    return cols <= 512;
+}
+
+}  // namespace
+
+bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* idx, void* o, int* status, cudaStream_t stream) {
+    StackPlan p;
+    if (!make_stack_plan(g, &p)) return BRA_ERR_UNSUPPORTED;
+    CUtensorMap tq, tk, tv;
+    if (!encode_region_map(&tq, q, g.B, g.H, g.W, g.C, g.ws, g.hs) ||
+        !encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs) ||
+        !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.ws, g.hs))
+        return BRA_ERR_UNSUPPORTED;
+    const int sms = sm_count();
+    if (sms <= 0) return BRA_ERR_CUDA;
+    const int grid = p.tiles < sms ? p.tiles : sms;
+    auto kernel = p.wgs == 2 ? (p.kn == 64 ? bra_attend_stack_kernel<2, true> : bra_attend_stack_kernel<2, false>)
+                             : (p.kn == 64 ? bra_attend_stack_kernel<1, true> : bra_attend_stack_kernel<1, false>);
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes) !=
+        cudaSuccess)
+        return BRA_ERR_CUDA;
+    const cudaError_t e = launch_after_previous(kernel, dim3(grid), dim3(32 * kCtrl + 128 * p.wgs), p.smem_bytes,
+                                                stream, tq, tk, tv, idx, static_cast<__nv_bfloat16*>(o), g,
+                                                p, status);
+    return e == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
+}  // namespace bra

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "../../include/bra.h"
@@ -42,8 +43,9 @@ bra_status make_geometry(const bra_shape* s, Geometry* g) {
     if (g->d != 32) return BRA_ERR_UNSUPPORTED;
     if (g->R > kMaxRegions) return BRA_ERR_UNSUPPORTED;
     if (s->heads > 65535) return BRA_ERR_UNSUPPORTED;
-    // pool: one 16-byte vector column per thread must cover C
+    // pool: the 16-byte channel vectors of one token must fit the CTA's threads
     if ((size_t)s->C * elem_bytes(s->dtype) > 16u * kPoolThreads) return BRA_ERR_UNSUPPORTED;
+    if ((int64_t)s->B * s->heads > 0x7fffffff) return BRA_ERR_UNSUPPORTED;
     return BRA_OK;
 }
 
@@ -64,6 +66,23 @@ Workspace carve(const Geometry& g, void* ws) {
             reinterpret_cast<int*>(base + 2 * mb)};
 }
 
+// Attention kernel selection.  The environment variable BRA_ATTEND_KERNEL
+// (read on every call) pins one kernel for testing: "stack" (persistent
+// tcgen05, regions of 16..64 tokens), "tiled" (tcgen05 per 128-query tile),
+// "simt" (CUDA cores); a pinned kernel that does not cover the shape makes
+// the call return BRA_ERR_UNSUPPORTED.  Unset or "auto": the first of those
+// that covers the shape (tensor-core kernels for bf16 only).
+enum class AttendKernel { kAuto, kStack, kTiled, kSimt };
+
+AttendKernel attend_kernel_choice() {
+    const char* e = getenv("BRA_ATTEND_KERNEL");
+    if (!e) return AttendKernel::kAuto;
+    if (!strcmp(e, "stack")) return AttendKernel::kStack;
+    if (!strcmp(e, "tiled")) return AttendKernel::kTiled;
+    if (!strcmp(e, "simt")) return AttendKernel::kSimt;
+    return AttendKernel::kAuto;
+}
+
 bra_status route_impl(const bra_shape* s, const Geometry& g, const void* q, const void* k,
                       int32_t* idx, const Workspace& w, cudaStream_t st) {
     if (g.B == 0) return BRA_OK;
@@ -78,10 +97,16 @@ bra_status attend_impl(const bra_shape* s, const Geometry& g, const void* q, con
                        cudaStream_t st) {
     if (g.B == 0) return BRA_OK;
     const bool bf16 = s->dtype == BRA_DTYPE_BF16;
-    if (bf16) {
-        const bra_status tc = attend_tc_launch(g, q, k, v, idx, o, w.status, st);
-        if (tc != BRA_ERR_UNSUPPORTED) return tc;
+    const AttendKernel choice = attend_kernel_choice();
+    if (bf16 && (choice == AttendKernel::kAuto || choice == AttendKernel::kStack)) {
+        const bra_status rc = attend_stack_launch(g, q, k, v, idx, o, w.status, st);
+        if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kStack) return rc;
     }
+    if (bf16 && (choice == AttendKernel::kAuto || choice == AttendKernel::kTiled)) {
+        const bra_status rc = attend_tc_launch(g, q, k, v, idx, o, w.status, st);
+        if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kTiled) return rc;
+    }
+    if (choice == AttendKernel::kStack || choice == AttendKernel::kTiled) return BRA_ERR_UNSUPPORTED;
     if ((int64_t)g.R * simt_plan(g).chunks > 0x7fffffff) return BRA_ERR_UNSUPPORTED;
     if (launch_attend_simt(bf16, q, k, v, idx, o, g, w.status, st) != cudaSuccess)
         return BRA_ERR_CUDA;

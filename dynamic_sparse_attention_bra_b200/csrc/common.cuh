@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace bra {
 
 // Geometry of one call, derived on the host from bra_shape.
@@ -56,6 +58,38 @@ __device__ __forceinline__ size_t token_offset(const Geometry& g, int b, int r, 
     const int ty = t / g.ws, tx = t - ty * g.ws;
     const size_t y = (size_t)ri * g.hs + ty, x = (size_t)rj * g.ws + tx;
     return (((size_t)b * g.H + y) * g.W + x) * g.C;
+}
+
+}  // namespace bra
+
+namespace bra {
+
+// Programmatic dependent launch: a kernel launched with
+// launch_after_previous() may start while the previous kernel on the stream
+// is finishing; it must call grid_dependency_wait() before touching anything
+// the previous kernel writes or reads.  A kernel calls allow_dependents()
+// once the kernel after it may begin its own set-up.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after_previous(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace bra

@@ -5,7 +5,8 @@
 
 namespace bra {
 
-constexpr int kPoolThreads = 256;
+constexpr int kPoolThreads = 128;
+constexpr int kStripMaxThreads = 512;
 constexpr int kRouteThreads = 256;
 constexpr int kMaxRegions = 256;   // S * S limit: 8 affinity columns per lane
 constexpr int kSimtThreads = 128;

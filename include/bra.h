@@ -36,7 +36,8 @@
  *    legacy default stream).  Arguments are checked on the host first; an
  *    invalid call returns an error and launches nothing.
  *  - Supported sizes: H % S == 0, W % S == 0, C % heads == 0, 1 <= topk <=
- *    S*S, S*S <= 256, d == 32, B >= 0 (B == 0 or an empty map is a no-op).
+ *    S*S, S*S <= 256, d == 32, C * sizeof(dtype) <= 2048 bytes (up to 32
+ *    bf16 or 16 fp32 heads), B >= 0 (B == 0 is a no-op).
  *    Pointers must be 16-byte aligned.  The S constraint is the pages'
  *    own (blog Part 3: S is chosen as a divisor of the map size so that no
  *    padding is needed); d == 32 is the head size of every BiFormer stage.
@@ -105,7 +106,9 @@ bra_status bra_route(const bra_shape* shape, const void* q, const void* k, int32
  * routed K/V tiles are staged in shared memory and never written to HBM.
  *   q, k, v    device, [B, H, W, C] of ``shape->dtype``, read only
  *   idx        device int32 [B, heads, S*S, topk], read only; any routing
- *              (it need not come from bra_route); an entry outside [0, S*S)
+ *              (it need not come from bra_route); a region repeated within a
+ *              row counts once (attention runs over the union of the routed
+ *              regions' tokens); an entry outside [0, S*S)
  *              makes the kernel skip that region's outputs and record
  *              BRA_ERR_BAD_ROUTE in the workspace status block
  *   o          device, [B, H, W, C] of ``shape->dtype``, written

@@ -40,6 +40,32 @@ def test_workloads_full_size(name):
     check_case(shape, seed)
 
 
+@pytest.fixture
+def pinned_kernel(request, monkeypatch):
+    """Pins the attention kernel through BRA_ATTEND_KERNEL for one test."""
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", request.param)
+    return request.param
+
+
+# Every attention kernel on every shape it covers (the default run above uses
+# the first kernel that covers each shape).
+KERNEL_CASES = [(k, w) for k in ("stack", "tiled", "simt") for w in ("stage1", "stage2", "stage3", "highres")]
+
+
+@pytest.mark.parametrize("pinned_kernel,name", KERNEL_CASES, indirect=["pinned_kernel"],
+                         ids=[f"{k}-{w}" for k, w in KERNEL_CASES])
+def test_each_kernel_on_workloads(pinned_kernel, name):
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape, seed = bi.WORKLOADS[name]
+    try:
+        check_case(shape, seed)
+    except bra.BraError as e:
+        if e.status != bra.BRA_ERR_UNSUPPORTED:
+            raise
+        assert pinned_kernel != "simt"
+        pytest.skip(f"{pinned_kernel} does not cover {name}")
+
+
 EXTRA = {
     # name: (B, H, W, C, heads, S, topk, dtype)
     "ragged_bf16": (2, 24, 24, 64, 2, 4, 3, "bf16"),        # n = 36: partial tiles
@@ -102,6 +128,49 @@ def test_attend_with_given_routing():
     assert bra.bra_device_status(s, ws) == bra.BRA_OK
     o_ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx_or, shape.heads, shape.S)
     assert np.abs(o.float().cpu().numpy() - o_ref).max() <= TOL["bf16"]
+
+
+def masked_dense_reference(inp, idx, heads, S):
+    """Attention of each query over the union of its region's routed regions,
+    as a dense masked softmax in float64 (set semantics for repeated routes)."""
+    q, k, v = inp.q_f64, inp.k_f64, inp.v_f64
+    B, H, W, C = q.shape
+    d = C // heads
+    reg = bi.region_map(H, W, S).reshape(-1)
+    out = np.zeros_like(q).reshape(B, H * W, C)
+    for b in range(B):
+        for h in range(heads):
+            sl = slice(h * d, (h + 1) * d)
+            Q, K, V = (x[b].reshape(H * W, C)[:, sl] for x in (q, k, v))
+            s = Q @ K.T / np.sqrt(d)
+            allowed = np.zeros((S * S, S * S), dtype=bool)
+            for r in range(S * S):
+                allowed[r, idx[b, h, r]] = True
+            s = np.where(allowed[reg][:, reg], s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            out[b, :, sl] = (p / p.sum(axis=1, keepdims=True)) @ V
+    return out.reshape(B, H, W, C)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_repeated_routes_attend_the_union(dtype):
+    """A caller-given routing that repeats a region in a row: every routed
+    region's tokens count once (both the tensor-core and the fp32 kernel)."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape = bi.BraShape(1, 16, 16, 32, 1, 4, 3, dtype)
+    inp = bi.make_inputs(shape, 12)
+    rng = np.random.default_rng(0)
+    idx = rng.integers(0, 16, size=(1, 1, 16, 3)).astype(np.int32)
+    idx[0, 0, :4] = [[2, 2, 2], [5, 1, 5], [0, 0, 7], [9, 3, 3]]
+    q, k, v = device_inputs(inp)
+    s = bra.shape_for(1, 16, 16, 32, 1, 4, 3, dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+    bra.bra_attend(s, q, k, v, torch.from_numpy(idx).cuda(), o, ws)
+    assert bra.bra_device_status(s, ws) == bra.BRA_OK
+    ref = masked_dense_reference(inp, idx, 1, 4)
+    assert np.abs(o.float().cpu().numpy() - ref).max() <= TOL[dtype]
 
 
 @pytest.mark.parametrize("bad_value", [-1, 16, 1 << 30])
