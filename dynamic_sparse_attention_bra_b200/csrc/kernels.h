@@ -6,7 +6,7 @@
 namespace bra {
 
 constexpr int kPoolThreads = 128;
-constexpr int kStripMaxThreads = 512;
+constexpr int kPoolWarpThreads = 128;  // 4 regions per CTA in the warp form
 constexpr int kRouteThreads = 256;
 constexpr int kMaxRegions = 256;   // S * S limit: 8 affinity columns per lane
 constexpr int kSimtThreads = 128;
