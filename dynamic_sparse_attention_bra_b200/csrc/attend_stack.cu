@@ -17,19 +17,23 @@
 // ever read, and P is zero outside the windows (each P row only ever writes
 // its own window), so O_h = P_h V_h (M = 64, N = 32) needs no masking either.
 //
-// Roles (192 threads, one CTA per SM, tiles strided by the grid):
-//   warp 0     producer: reads the tile's routes, issues TMA box loads of the
-//              query regions and of every routed key/value region straight
-//              from the [B, H, W, C] maps into a ring of shared-memory stages
-//              (64-byte swizzle), completion counted on the stage's mbarrier;
-//   warp 1     one lane issues the MMAs: S = Q K^T for tile i + 1 (double
-//              buffered in TMEM) before P V for tile i;
-//   warps 2-5  softmax and epilogue, one query row per thread: read the row's
-//              window of S, base-2 softmax in fp32, P as bf16 into 128-byte
+// Roles (one CTA per SM, tiles strided by the grid):
+//   warps 0-1  producers, tiles alternating between them: read the tile's
+//              routes (prefetched into shared memory), then issue TMA box
+//              loads of the query regions and of every routed key/value
+//              region straight from the [B, H, W, C] maps into a ring of
+//              shared-memory stages (64-byte swizzle), completion counted on
+//              the stage's mbarrier;
+//   warp 2     one lane issues S = Q K^T for every tile as soon as it lands;
+//   warp 3     one lane issues O = P V (with the row sums of P) for every tile
+//              as soon as its P is written, then releases the stage;
+//   then 1, 2 or 4 softmax warp groups, one query row per thread: read the
+//              row's window of S, base-2 softmax, P as bf16 into 128-byte
 //              swizzled shared memory, then O = (P V) / l to global memory.
 // Every mbarrier wait is bounded; on expiry the kernel records
 // kDevTimeout, stops all roles, drains its MMAs and frees TMEM.
 #include <cuda.h>
+#include <stdlib.h>
 
 #include "attend_tc.h"
 #include "kernels.h"
@@ -44,7 +48,6 @@ constexpr int kMaxRoutes = 16;  // kn <= 256 with n >= 16
 constexpr int kMaxStages = 8;
 constexpr int kMaxSBuf = 8;
 constexpr uint32_t kWait = 1u << 22;
-constexpr uint32_t kSpinLimit = 1u << 26;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kSmemBudget = 227 * 1024;
 
@@ -61,6 +64,7 @@ struct StackPlan {
     int items;              // (slot, route) pairs of a tile: 2 * Gq * topk <= 32
     int wgs;                // softmax warp groups (1 or 2)
     int pdepth;             // P buffers per warp group (2: a tile's epilogue waits one tile)
+    int nprod;              // producer warps in use: min(kProd, stages)
     uint32_t stage_bytes;   // Q (2 x 64 rows) + K + V of one tile
     uint32_t k_off, v_off;  // offsets inside a stage
     uint32_t p_half;        // one half of a P buffer: ceil(N / 64) atoms of 64 rows x 128 B
@@ -77,6 +81,10 @@ struct TileMeta {
     uint32_t live[2][kMaxSlots];   // bit m: route m loaded (in range, first occurrence)
 };
 
+constexpr int kProd = 2;   // producer warps (tiles alternate between them)
+constexpr int kCtrl = kProd + 2;  // + the S issuer warp and the P V issuer warp
+constexpr int kRouteAhead = 4;    // tiles of routes a producer warp has in flight
+
 struct Barriers {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
@@ -84,6 +92,7 @@ struct Barriers {
     uint64_t p_full[4];
     uint64_t drain[2];
     TileMeta meta[kMaxStages];
+    int32_t routes[kProd][kRouteAhead][32];  // per producer warp: routes of its next tiles
     uint32_t tmem;
     int abort;
 };
@@ -110,13 +119,10 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
 // Per-row state kept from a tile's softmax until its epilogue.
 struct RowState {
     int region, b, h;
-    float l;
 };
 
-constexpr int kProd = 2;   // producer warps (tiles alternate between them)
-constexpr int kCtrl = kProd + 2;  // + the S issuer warp and the P V issuer warp
 
-// WGS softmax warp groups (1 or 2); KN64: every window is exactly 64 keys.
+// WGS softmax warp groups (1, 2 or 4); KN64: every window is exactly 64 keys.
 template <int WGS, bool KN64>
 __global__ void __launch_bounds__(32 * kCtrl + 128 * WGS, 1)
 bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -168,7 +174,6 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
     // Everything above overlaps the routing kernel; from here on the routes
     // are read and O is written.
     grid_dependency_wait();
-
     if (warp < kProd) {
         // ------------------------------------------------------------ producer
         // Producer warp w loads tiles w, w + kProd, ...  Lane j first owns item
@@ -177,8 +182,9 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
         // box per live item -- go out one box per lane in a single TMA
         // instruction (copies from one thread are processed in order, copies
         // from different lanes in parallel), rotated across tiles so that
-        // successive tiles use different lanes.  Routes of the warp's next tile
-        // are read while this tile's copies are issued.
+        // successive tiles use different lanes.  Routes reach shared memory by
+        // 4-byte asynchronous copies issued kRouteAhead of the warp's tiles
+        // early, so the route latency is paid once, not once per tile.
         if (lane == 0 && warp == 0) {
             ptx::tma_prefetch_desc(&tq);
             ptx::tma_prefetch_desc(&tk);
@@ -194,18 +200,38 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
         const uint32_t nbytes_region = (uint32_t)g.n * 64u;
         const int nq = 2 * p.Gq;                 // query boxes of a tile
         const int nboxes = nq + 2 * p.items;     // + key and value boxes
-        auto fetch = [&](int i, int& reg) -> int {
+        // Region of this lane's item in local tile i (-1: none), and the
+        // asynchronous fetch of its route into ring slot (i / kProd) % kRouteAhead;
+        // each fetch is one cp.async group, issued kRouteAhead tiles early.
+        auto item_region = [&](int i, int& bh) -> int {
             const int t = blockIdx.x + i * gridDim.x;
-            const int bh = t / p.tiles_bh, tt = t - bh * p.tiles_bh;
+            bh = t / p.tiles_bh;
+            const int tt = t - bh * p.tiles_bh;
             const int ht = tt * 2 + half;
             const int r = ht * p.Gq + slot;
-            reg = (item && ht < p.halves && r < g.R) ? r : -1;
-            return reg >= 0 ? __ldg(idx + ((size_t)bh * g.R + r) * g.topk + m) : 0;
+            return (item && ht < p.halves && r < g.R) ? r : -1;
         };
-        int cur_reg = -1, nxt_reg = -1;
-        int cur = warp < my_tiles ? fetch(warp, cur_reg) : 0;
-        for (int i = warp; i < my_tiles; i += kProd) {
-            const int nxt = i + kProd < my_tiles ? fetch(i + kProd, nxt_reg) : 0;
+        auto fetch = [&](int i) {
+            if (i < my_tiles) {
+                int bh = 0;
+                const int r = item_region(i, bh);
+                const int32_t* src = idx + ((size_t)bh * g.R + (r >= 0 ? r : 0)) * g.topk + m;
+                ptx::cp_async4(ptx::smem_addr(&sb->routes[warp][(i / p.nprod) % kRouteAhead][lane]), src,
+                               r >= 0 ? 4u : 0u);
+            }
+            ptx::cp_async_commit();  // an empty group past the last tile keeps the count uniform
+        };
+        // A stage's release k is awaited only after release k - 1 has happened
+        // (the wait is on its parity), which holds when each producer warp's
+        // previous tile used a stage released later: hence nprod <= stages.
+        if (warp < p.nprod)
+            for (int a = 0; a < kRouteAhead; ++a) fetch(warp + a * p.nprod);
+        for (int i = warp; warp < p.nprod && i < my_tiles; i += p.nprod) {
+            ptx::cp_async_wait_group<kRouteAhead - 1>();  // this tile's routes have landed
+            int bh_unused = 0;
+            const int cur_reg = item_region(i, bh_unused);
+            const int cur = sb->routes[warp][(i / p.nprod) % kRouteAhead][lane];
+            fetch(i + kRouteAhead * p.nprod);  // reuses the slot just read
             const int s = i % p.stages;
             if (i >= p.stages && !wait_or_abort(&sb->empty[s], ((i / p.stages) - 1) & 1, sb, status))
                 break;
@@ -238,7 +264,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             if (lane == 0) ptx::mbar_arrive_expect_tx(&sb->full[s], bytes);
             __syncwarp();
             const uint32_t stage = sbase + (uint32_t)s * p.stage_bytes;
-            const int rot = (i / kProd * nboxes) & 31;
+            const int rot = (i / p.nprod * nboxes) & 31;
             for (int j0 = 0; j0 < nboxes; j0 += 32) {
                 const int j = j0 + ((lane - rot) & 31);  // box this lane issues
                 // the item behind box j: query box j -> slot lane (j * topk), K/V box -> item
@@ -262,9 +288,8 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                                      hd * 32, qj * g.ws, qi * g.hs, b, &sb->full[s]);
                 }
             }
-            cur = nxt;
-            cur_reg = nxt_reg;
         }
+        ptx::cp_async_wait_all();
     } else if (warp == kProd) {
         // ------------------------------------------------------- S = Q K^T issuer
         // One lane issues S for every tile in order as soon as the tile's stage
@@ -316,7 +341,6 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                         const uint32_t d = tmem + sbuf * p.N + ((uint32_t)(half * 16) << 16);
                         const uint64_t a = ptx::smem_desc(pbase + half * p.p_half + (kk >> 2) * 8192 + (kk & 3) * 32,
                                                           16, 1024, ptx::kSwizzle128B);
-                        // B: V rows (N 0..31) and, one leading-byte offset further, the ones (N 32..63)
                         const uint32_t vaddr = stage + p.v_off + (uint32_t)half * p.N * 64 + kk * 1024;
                         const uint64_t bd = ptx::smem_desc(vaddr, ones + kk * 1024 - vaddr, 512, ptx::kSwizzle64B);
                         ptx::mma_bf16(d, a, bd, idesc_pv, kk);
@@ -349,35 +373,43 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             const int sbuf = j % p.nsb;
             if (!wait_or_abort(&sb->o_full[sbuf], (j / p.nsb) & 1, sb, status)) return false;
             ptx::tc_fence_after();
-            uint32_t r[32], rl[16];
-            float l = 0.f;
+            // l (column 32) with O columns 0-15, then O columns 16-31: no more
+            // than 17 accumulator words are held at a time.
+            uint32_t r[16], lw = 0;
             if (slot_ok) {
-                ptx::tmem_ld32(tmem + lane_addr + sbuf * p.N, r);
-                ptx::tmem_ld16(tmem + lane_addr + sbuf * p.N + 32, rl);
-                ptx::tmem_ld_wait();
-                l = __uint_as_float(rl[0]);
+                ptx::tmem_ld16(tmem + lane_addr + sbuf * p.N, r);
+                lw = ptx::tmem_ld1(tmem + lane_addr + sbuf * p.N + 32);
+                ptx::tmem_wait17(r, lw);
+            }
+            const float l = __uint_as_float(lw);
+            const bool write = st.region >= 0 && l > 0.f;
+            const float inv = write ? 1.f / l : 0.f;
+            int4* dst = write ? reinterpret_cast<int4*>(o + token_offset(g, st.b, st.region, tok) + (size_t)st.h * 32)
+                              : nullptr;
+#pragma unroll
+            for (int h16 = 0; h16 < 2; ++h16) {
+                if (h16 == 1 && slot_ok) {
+                    ptx::tmem_ld16(tmem + lane_addr + sbuf * p.N + 16, r);
+                    ptx::tmem_wait16(r);
+                }
+                if (write) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = ptx::pack_bf16x2(__uint_as_float(r[8 * c + 2 * e]) * inv,
+                                                    __uint_as_float(r[8 * c + 2 * e + 1]) * inv);
+                        __stcs(dst + 2 * h16 + c, make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]));  // streamed: O is not re-read
+                    }
+                }
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&sb->s_free[sbuf]);
-            if (st.region >= 0 && l > 0.f) {
-                const float inv = 1.f / l;
-                int4* dst = reinterpret_cast<int4*>(o + token_offset(g, st.b, st.region, tok) + (size_t)st.h * 32);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[8 * c + 2 * e]) * inv,
-                                                                        __uint_as_float(r[8 * c + 2 * e + 1]) * inv);
-                        w[e] = *reinterpret_cast<const uint32_t*>(&pr);
-                    }
-                    __stcs(dst + c, make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]));  // streamed: O is not re-read
-                }
-            }
             return true;
         };
 
-        RowState prev = {-1, 0, 0, 0.f};
+        RowState prev = {-1, 0, 0};
         bool ok = true;
         int last = -1;
         for (int i = wg; ok && i < my_tiles; i += WGS) {
@@ -392,97 +424,88 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             cur.h = M.h;
             const uint32_t live = slot_ok ? M.live[half][slot] : 0u;
             const bool all_live = live == full_live;
-            float l = 0.f;
             if (slot_ok) {
                 const uint32_t col0 = sbuf * p.N + slot * p.kn;
                 const uint32_t prow = sbase + p.p_off + (uint32_t)pb * 2u * p.p_half + half * p.p_half + m * 128;
-                // segment j (16 columns) of the window belongs to route j * 16 / n
-                auto seg_mask = [&](int c) -> uint32_t {
-                    if (all_live) return 0xffffffffu;
-                    const int r0 = (c >> 4) * 16 / g.n, r1 = ((c >> 4) + 1) * 16 / g.n;
-                    return (((live >> r0) & 1u) ? 0x0000ffffu : 0u) | (((live >> r1) & 1u) ? 0xffff0000u : 0u);
-                };
-                auto write_p = [&](int c, const uint32_t* packed) {
+                // 16 p values of window columns c .. c + 15 as 8 bf16 pairs: two
+                // 16-byte chunks of the row's 128-byte swizzled atom line.
+                auto write_p16 = [&](int c, const uint32_t* packed) {
                     const int col = slot * p.kn + c;  // window column inside the half's P
                     const uint32_t atom = prow + (uint32_t)(col >> 6) * 8192u;
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < 2; ++cc) {
                         const int chunk = ((col & 63) >> 3) + cc;
                         ptx::st_shared_v4(atom + ((chunk ^ (m & 7)) << 4), packed[4 * cc], packed[4 * cc + 1],
                                           packed[4 * cc + 2], packed[4 * cc + 3]);
                     }
                 };
-                // p for 32 scores of chunk c (fp32 exponentials, rounded to bf16)
-                auto exp_chunk = [&](const uint32_t* r, uint32_t km, float msl, uint32_t* packed) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ((km >> (2 * e)) & 1u) ? ptx::ex2(fmaf(__uint_as_float(r[2 * e]), sl, -msl)) : 0.f;
-                        const float p1 = ((km >> (2 * e + 1)) & 1u) ? ptx::ex2(fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)) : 0.f;
-                        const __nv_bfloat162 pbf = __floats2bfloat162_rn(p0, p1);
-                        packed[e] = *reinterpret_cast<const uint32_t*>(&pbf);
-                    }
-                };
                 if (KN64 && __all_sync(0xffffffffu, all_live)) {
                     // Every route of every row of this warp is live: no masks.
-                    // Two 32-column TMEM reads for the max, two more for p, so no
-                    // more than 32 scores are live in registers at a time.
+                    // TMEM is read 16 columns at a time (max pass, then p pass),
+                    // each read waited on before the next is issued.
                     float m8[8];
-                    {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tmem + lane_addr + col0, r);
-                        ptx::tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(r[e]);
+                    for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
-                        for (int e = 8; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(r[e]));
-                        ptx::tmem_ld32(tmem + lane_addr + col0 + 32, r);
-                        ptx::tmem_ld_wait();
+                    for (int c = 0; c < 64; c += 16) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_wait16(r);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(r[e]));
+                        for (int e = 0; e < 16; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(r[e]));
                     }
                     const float msl = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl;
                     // p = 2^(s * sl - max) on bf16 pairs: P enters the MMA as bf16
                     // anyway, and the row sums come from the same bf16 values (P x ones).
 #pragma unroll
-                    for (int c = 0; c < 64; c += 32) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tmem + lane_addr + col0 + c, r);
-                        ptx::tmem_ld_wait();
-                        uint32_t packed[16];
+                    for (int c = 0; c < 64; c += 16) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_wait16(r);
+                        uint32_t packed[8];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
+                        for (int e = 0; e < 8; ++e)
                             packed[e] = ptx::ex2_bf16x2(ptx::pack_bf16x2(fmaf(__uint_as_float(r[2 * e]), sl, -msl),
                                                                          fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)));
-                        write_p(c, packed);
+                        write_p16(c, packed);
                     }
                 } else {
+                    // 16-column segment c / 16 of the window belongs to route c * 16 / n
+                    // (n is a multiple of 16); a dead route's scores are skipped.
+                    auto seg_live = [&](int c) -> bool { return (live >> ((c >> 4) * 16 / g.n)) & 1u; };
                     float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    for (int c = 0; c < p.kn; c += 32) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tmem + lane_addr + col0 + c, r);
-                        ptx::tmem_ld_wait();
-                        const uint32_t km = seg_mask(c);
+                    for (int c = 0; c < p.kn; c += 16) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_wait16(r);
+                        if (seg_live(c)) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            m4[e & 3] = fmaxf(m4[e & 3], ((km >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY);
+                            for (int e = 0; e < 16; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(r[e]));
+                        }
                     }
                     const float msl = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
-                    for (int c = 0; c < p.kn; c += 32) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tmem + lane_addr + col0 + c, r);
-                        ptx::tmem_ld_wait();
-                        uint32_t packed[16];
-                        exp_chunk(r, seg_mask(c), msl, packed);
-                        write_p(c, packed);
+                    for (int c = 0; c < p.kn; c += 16) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(tmem + lane_addr + col0 + c, r);
+                        ptx::tmem_wait16(r);
+                        const bool on = seg_live(c);
+                        uint32_t packed[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            // fp32 exponentials, rounded to bf16
+                            const float p0 = on ? ptx::ex2(fmaf(__uint_as_float(r[2 * e]), sl, -msl)) : 0.f;
+                            const float p1 = on ? ptx::ex2(fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)) : 0.f;
+                            packed[e] = ptx::pack_bf16x2(p0, p1);
+                        }
+                        write_p16(c, packed);
                     }
                 }
             }
-            cur.l = l;
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&sb->p_full[pb]);
-            if (p.pdepth == 2) {
+            if (WGS < 4 && p.pdepth == 2) {  // four groups always run one P buffer each
                 // This group's previous tile finishes while this tile's P V runs.
                 if (last >= 0) ok = epilogue(last, prev);
                 prev = cur;
@@ -502,7 +525,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
     }
 }
 
-bool make_stack_plan(const Geometry& g, StackPlan* p) {
+bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     if (g.d != 32 || g.n % 16 != 0 || g.n > 64) return false;
     const int kn = g.topk * g.n;
     if (kn > 256 || kn % 32 != 0 || g.topk > kMaxRoutes) return false;
@@ -527,18 +550,24 @@ bool make_stack_plan(const Geometry& g, StackPlan* p) {
     p->p_half = (uint32_t)((p->N + 63) / 64) * 8192u;
     const uint32_t misc = (uint32_t)((sizeof(Barriers) + 1023) / 1024 * 1024);
     const uint32_t ones_bytes = (uint32_t)p->N * 64u;  // N keys x 64 B of bf16 ones
+    if (512 / p->N < 2) return false;
+    p->nsb = 512 / p->N >= kMaxSBuf ? kMaxSBuf : 512 / p->N;
     // Softmax warp groups x P buffers per group, most overlap first, as long
-    // as a load ring of at least 3 stages (2 for the last option) remains.
-    static const int kOptions[4][2] = {{2, 2}, {2, 1}, {1, 2}, {1, 1}};
+    // as the load ring keeps enough stages to feed that many groups.  Waits
+    // on a barrier's parity need the barrier's previous phase complete: a
+    // group's earlier tiles must cover the tile `stages` (and `nsb`) before,
+    // so groups <= stages and nsb a multiple of the groups.
+    static const int kOptions[5][3] = {{4, 1, 5}, {2, 2, 3}, {2, 1, 3}, {1, 2, 3}, {1, 1, 2}};
     int stages = 0;
     bool found = false;
-    for (int o = 0; o < 4 && !found; ++o) {
+    for (int o = 0; o < 5 && !found; ++o) {
+        if (kOptions[o][0] > max_groups || p->nsb % kOptions[o][0] != 0) continue;
         p->wgs = kOptions[o][0];
         p->pdepth = kOptions[o][1];
         p->np = p->wgs * p->pdepth;
         const uint32_t used = 1024 + misc + ones_bytes + (uint32_t)p->np * 2u * p->p_half;
         stages = used < kSmemBudget ? (int)((kSmemBudget - used) / p->stage_bytes) : 0;
-        found = stages >= (o == 3 ? 2 : 3);
+        found = stages >= kOptions[o][2] && stages >= p->wgs;
     }
     if (!found) return false;
     if (stages > kMaxStages) stages = kMaxStages;
@@ -547,8 +576,7 @@ bool make_stack_plan(const Geometry& g, StackPlan* p) {
     p->ones_off = p->p_off + (uint32_t)p->np * 2u * p->p_half;
     p->bar_off = p->ones_off + ones_bytes;
     p->smem_bytes = p->bar_off + (uint32_t)sizeof(Barriers) + 1024;
-    if (512 / p->N < 2) return false;
-    p->nsb = 512 / p->N >= kMaxSBuf ? kMaxSBuf : 512 / p->N;
+    p->nprod = stages < kProd ? stages : kProd;
     uint32_t cols = 32;
     while (cols < (uint32_t)(p->nsb * p->N)) cols <<= 1;
     p->tmem_cols = cols;
@@ -559,8 +587,14 @@ bool make_stack_plan(const Geometry& g, StackPlan* p) {
 
 bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* idx, void* o, int* status, cudaStream_t stream) {
+    // BRA_STACK_GROUPS caps the softmax warp groups (1, 2 or 4; default 4).
+    int max_groups = 4;
+    if (const char* env = getenv("BRA_STACK_GROUPS")) {
+        const int v = atoi(env);
+        if (v >= 1 && v <= 4) max_groups = v;
+    }
     StackPlan p;
-    if (!make_stack_plan(g, &p)) return BRA_ERR_UNSUPPORTED;
+    if (!make_stack_plan(g, max_groups, &p)) return BRA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv;
     if (!encode_region_map(&tq, q, g.B, g.H, g.W, g.C, g.ws, g.hs) ||
         !encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs) ||
@@ -569,8 +603,9 @@ bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, 
     const int sms = sm_count();
     if (sms <= 0) return BRA_ERR_CUDA;
     const int grid = p.tiles < sms ? p.tiles : sms;
-    auto kernel = p.wgs == 2 ? (p.kn == 64 ? bra_attend_stack_kernel<2, true> : bra_attend_stack_kernel<2, false>)
-                             : (p.kn == 64 ? bra_attend_stack_kernel<1, true> : bra_attend_stack_kernel<1, false>);
+    auto kernel = p.wgs == 4   ? (p.kn == 64 ? bra_attend_stack_kernel<4, true> : bra_attend_stack_kernel<4, false>)
+                  : p.wgs == 2 ? (p.kn == 64 ? bra_attend_stack_kernel<2, true> : bra_attend_stack_kernel<2, false>)
+                               : (p.kn == 64 ? bra_attend_stack_kernel<1, true> : bra_attend_stack_kernel<1, false>);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes) !=
         cudaSuccess)
         return BRA_ERR_CUDA;

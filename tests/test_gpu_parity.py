@@ -72,6 +72,7 @@ EXTRA = {
     "ragged_f32": (2, 24, 24, 64, 2, 4, 3, "f32"),
     "nonsquare_regions": (1, 18, 12, 32, 1, 6, 5, "bf16"),  # 3x2 tokens per region
     "wide_map": (1, 16, 48, 64, 2, 4, 2, "bf16"),           # 4x12 tokens per region
+    "wide_map_batch": (24, 16, 48, 64, 2, 4, 2, "bf16"),    # the same, several tiles per CTA
     "dense_topk": (1, 16, 16, 64, 2, 4, 16, "bf16"),        # k = S^2: full attention
     "single_region": (2, 16, 20, 64, 2, 1, 1, "bf16"),      # n = 320: several query tiles
     "single_token_regions": (2, 8, 8, 64, 2, 8, 4, "bf16"), # n = 1
@@ -201,3 +202,21 @@ def test_empty_batch_is_a_noop():
     idx = torch.zeros(4, dtype=torch.int32, device="cuda")
     bra.bra_forward(s, buf, buf, buf, buf, idx, ws)
     assert bra.bra_device_status(s, ws) == bra.BRA_OK
+
+
+# The persistent kernel with each number of softmax warp groups (1, 2, 4) on
+# the shapes it covers: 64-key windows with one and with four query regions
+# per half, and 96-key windows (the masked softmax path).
+GROUP_CASES = [(gr, w) for gr in (1, 2, 4) for w in ("stage1", "stage2", "wide_map_batch")]
+
+
+@pytest.mark.parametrize("groups,name", GROUP_CASES, ids=[f"groups{g}-{w}" for g, w in GROUP_CASES])
+def test_stack_kernel_groups(groups, name, monkeypatch):
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", "stack")
+    monkeypatch.setenv("BRA_STACK_GROUPS", str(groups))
+    if name in bi.WORKLOADS:
+        shape, seed = bi.WORKLOADS[name]
+    else:
+        B, H, W, C, heads, S, topk, dtype = EXTRA[name]
+        shape, seed = bi.BraShape(B, H, W, C, heads, S, topk, dtype), 11
+    check_case(shape, seed)
