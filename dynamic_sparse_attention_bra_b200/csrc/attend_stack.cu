@@ -3,8 +3,13 @@
 // section 2.2, step 4: gather the routed key-value regions, then token
 // attention over them).
 //
-// Tiling.  A tile is 128 query rows of one (batch, head) split into two
-// 64-row halves; a half holds Gq whole query regions (Gq * n <= 64).  Each
+// Tiling.  A tile is two 64-row halves; a half holds Gq whole query regions
+// (Gq * n <= 64) of one (batch, head).  With an even number of heads the two
+// halves are the heads 2j and 2j + 1 of the same regions (head pairing): the
+// query tokens then arrive as one 128-byte-row box per region (both heads'
+// 64 channels, 128-byte swizzle) and each half's Q K^T reads its own 64-byte
+// column range of those rows; otherwise the halves are consecutive region
+// groups of one head with 64-byte query rows.  Each
 // query region r brings its own key list: the tokens of its routed regions
 // I^r[r][0..topk), kn = topk * n keys, stacked slot after slot, so half h
 // multiplies Q_h [64 x 32] by K_h^T [32 x Gq*kn] with one M = 64 tcgen05.mma
@@ -55,8 +60,9 @@ struct StackPlan {
     int Gq;                 // query regions per half
     int kn;                 // keys per query region
     int N;                  // keys per half = Gq * kn (MMA N of Q K^T)
-    int halves;             // half tiles per (batch, head)
-    int tiles_bh;           // tiles per (batch, head)
+    int hp;                 // 1: halves are a head pair (heads even), 0: region groups of one head
+    int halves;             // region groups (of Gq regions) per (batch, head)
+    int tiles_bh;           // tiles per (batch, head) or, head-paired, per (batch, head pair)
     int tiles;              // all tiles
     int stages;             // shared-memory ring depth
     int nsb;                // S buffers in TMEM
@@ -76,7 +82,7 @@ struct StackPlan {
 };
 
 struct TileMeta {
-    int b, h;
+    int b, h[2];                   // batch, head of each half
     int reg[2][kMaxSlots];         // query region of each slot, -1 if none
     uint32_t live[2][kMaxSlots];   // bit m: route m loaded (in range, first occurrence)
 };
@@ -197,17 +203,26 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
         const int m = item ? lane % g.topk : 0;
         const int lane0 = lane - m;  // lane of route 0 of this slot
         const uint32_t slot_lanes = (g.topk >= 32 ? 0xffffffffu : ((1u << g.topk) - 1u)) << lane0;
-        const uint32_t nbytes_region = (uint32_t)g.n * 64u;
-        const int nq = 2 * p.Gq;                 // query boxes of a tile
-        const int nboxes = nq + 2 * p.items;     // + key and value boxes
+        const uint32_t nbytes_region = (uint32_t)g.n * 64u;        // one head of a region
+        const int nq = p.hp ? p.Gq : 2 * p.Gq;                     // query boxes of a tile
+        const uint32_t qbytes_box = p.hp ? 2u * nbytes_region : nbytes_region;
+        const int nboxes = nq + 2 * p.items;                       // + key and value boxes
         // Region of this lane's item in local tile i (-1: none), and the
         // asynchronous fetch of its route into ring slot (i / kProd) % kRouteAhead;
         // each fetch is one cp.async group, issued kRouteAhead tiles early.
+        // (batch, head) slice of half hf of tile t and the tile's region group
+        auto tile_slice = [&](int t, int hf, int& ht) -> int {
+            const int u = t / p.tiles_bh, tt = t - u * p.tiles_bh;
+            if (p.hp) {
+                ht = tt;
+                return 2 * u + hf;  // u = b * heads / 2 + head pair; b * heads + 2 * pair + hf
+            }
+            ht = tt * 2 + hf;
+            return u;
+        };
         auto item_region = [&](int i, int& bh) -> int {
-            const int t = blockIdx.x + i * gridDim.x;
-            bh = t / p.tiles_bh;
-            const int tt = t - bh * p.tiles_bh;
-            const int ht = tt * 2 + half;
+            int ht = 0;
+            bh = tile_slice(blockIdx.x + i * gridDim.x, half, ht);
             const int r = ht * p.Gq + slot;
             return (item && ht < p.halves && r < g.R) ? r : -1;
         };
@@ -236,8 +251,10 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             if (i >= p.stages && !wait_or_abort(&sb->empty[s], ((i / p.stages) - 1) & 1, sb, status))
                 break;
             const int t = blockIdx.x + i * gridDim.x;
-            const int bh = t / p.tiles_bh;
-            const int b = bh / g.heads, hd = bh - b * g.heads;
+            int ht0 = 0;
+            const int bh0 = tile_slice(t, 0, ht0);  // half 0; half 1 is the next head or the same
+            const int b = bh0 / g.heads, hd0 = bh0 - b * g.heads;
+            const int hd1 = p.hp ? hd0 + 1 : hd0;
             const bool valid = cur_reg >= 0;
             const uint32_t bad = __ballot_sync(0xffffffffu, valid && (cur < 0 || cur >= g.R));
             const bool slot_ok = valid && !(bad & slot_lanes);
@@ -250,6 +267,9 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             const bool live = slot_ok && !dup;
             const uint32_t live_lanes = __ballot_sync(0xffffffffu, live);
             const uint32_t ok_lanes = __ballot_sync(0xffffffffu, slot_ok && m == 0);
+            // query boxes: per (half, slot) with a usable route set, or, head-paired,
+            // per slot whose region exists (one box serves both halves)
+            const uint32_t q_lanes = p.hp ? __ballot_sync(0xffffffffu, valid && half == 0 && m == 0) : ok_lanes;
             TileMeta& M = sb->meta[s];
             if (item && m == 0) {
                 M.reg[half][slot] = slot_ok ? cur_reg : -1;
@@ -257,9 +277,10 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             }
             if (lane == 0) {
                 M.b = b;
-                M.h = hd;
+                M.h[0] = hd0;
+                M.h[1] = hd1;
             }
-            const uint32_t bytes = (uint32_t)(__popc(ok_lanes) + 2 * __popc(live_lanes)) * nbytes_region;
+            const uint32_t bytes = (uint32_t)__popc(q_lanes) * qbytes_box + 2u * __popc(live_lanes) * nbytes_region;
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_expect_tx(&sb->full[s], bytes);
             __syncwarp();
@@ -275,17 +296,20 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 if (j >= nboxes) continue;
                 const int x_half = it / per_half, x_slot = (it / g.topk) % p.Gq, x_m = it % g.topk;
                 if (j < nq) {
-                    if ((ok_lanes >> it) & 1u) {
+                    if ((q_lanes >> it) & 1u) {
                         const int ri = x_reg / g.S, rj = x_reg - ri * g.S;
-                        ptx::tma_load_4d(stage + x_half * 4096 + x_slot * nbytes_region, &tq, hd * 32, rj * g.ws,
-                                         ri * g.hs, b, &sb->full[s]);
+                        // head-paired: 64 channels (heads hd0, hd0 + 1) of the slot's region
+                        const uint32_t qoff = p.hp ? (uint32_t)x_slot * qbytes_box
+                                                   : (uint32_t)x_half * 4096u + (uint32_t)x_slot * nbytes_region;
+                        ptx::tma_load_4d(stage + qoff, &tq, (x_half ? hd1 : hd0) * 32, rj * g.ws, ri * g.hs, b,
+                                         &sb->full[s]);
                     }
                 } else if ((live_lanes >> it) & 1u) {
                     const int qi = x_cur / g.S, qj = x_cur - qi * g.S;
                     const uint32_t koff = (uint32_t)(x_half * p.N + x_slot * p.kn + x_m * g.n) * 64u;
                     const bool is_v = (j - nq) & 1;
                     ptx::tma_load_4d(stage + (is_v ? p.v_off : p.k_off) + koff, is_v ? (const void*)&tv : (const void*)&tk,
-                                     hd * 32, qj * g.ws, qi * g.hs, b, &sb->full[s]);
+                                     (x_half ? hd1 : hd0) * 32, qj * g.ws, qi * g.hs, b, &sb->full[s]);
                 }
             }
         }
@@ -307,7 +331,10 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 for (int kk = 0; kk < 2; ++kk) {
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
-                        const uint64_t a = ptx::smem_desc(stage + half * 4096 + kk * 32, 16, 512, ptx::kSwizzle64B);
+                        // A: head-paired, 128-byte rows of both heads (half h at byte 64 h);
+                        // otherwise 64-byte rows, one half after the other
+                        const uint64_t a = p.hp ? ptx::smem_desc(stage + half * 64 + kk * 32, 16, 1024, ptx::kSwizzle128B)
+                                                : ptx::smem_desc(stage + half * 4096 + kk * 32, 16, 512, ptx::kSwizzle64B);
                         const uint64_t bd = ptx::smem_desc(stage + p.k_off + (uint32_t)half * p.N * 64 + kk * 32, 16,
                                                            512, ptx::kSwizzle64B);
                         ptx::mma_bf16(tmem + sbuf * p.N + ((uint32_t)(half * 16) << 16), a, bd, idesc_qk, kk);
@@ -421,7 +448,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             RowState cur;
             cur.region = slot_ok ? M.reg[half][slot] : -1;
             cur.b = M.b;
-            cur.h = M.h;
+            cur.h = M.h[half];
             const uint32_t live = slot_ok ? M.live[half][slot] : 0u;
             const bool all_live = live == full_live;
             if (slot_ok) {
@@ -538,9 +565,10 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     if (p->items > 32) return false;
     p->N = p->Gq * kn;
     if (p->N < 64) return false;  // the O block (32 columns) and its row sums (16) reuse S
+    p->hp = g.heads % 2 == 0 ? 1 : 0;
     p->halves = (g.R + p->Gq - 1) / p->Gq;
-    p->tiles_bh = (p->halves + 1) / 2;
-    const long long tiles = (long long)g.B * g.heads * p->tiles_bh;
+    p->tiles_bh = p->hp ? p->halves : (p->halves + 1) / 2;
+    const long long tiles = (long long)g.B * (p->hp ? g.heads / 2 : g.heads) * p->tiles_bh;
     if (tiles > 0x7fffffffLL) return false;
     p->tiles = (int)tiles;
     const uint32_t kv = (uint32_t)2 * p->N * 64;  // two halves of N rows of 64 B
@@ -596,9 +624,9 @@ bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, 
     StackPlan p;
     if (!make_stack_plan(g, max_groups, &p)) return BRA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv;
-    if (!encode_region_map(&tq, q, g.B, g.H, g.W, g.C, g.ws, g.hs) ||
-        !encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs) ||
-        !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.ws, g.hs))
+    if (!encode_region_map(&tq, q, g.B, g.H, g.W, g.C, g.ws, g.hs, p.hp ? 64 : 32) ||
+        !encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs, 32) ||
+        !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.ws, g.hs, 32))
         return BRA_ERR_UNSUPPORTED;
     const int sms = sm_count();
     if (sms <= 0) return BRA_ERR_CUDA;

@@ -7,11 +7,12 @@
 
 namespace bra {
 
-// Tensor map whose box is one head (32 channels) of a box_w x box_h block of
-// tokens of one image, 64-byte swizzled in shared memory.  Returns false if
-// the driver entry point is missing or the encoder rejects the map.
+// Tensor map whose box is box_c channels (32: one head, 64-byte swizzle in
+// shared memory; 64: two heads, 128-byte swizzle) of a box_w x box_h block of
+// tokens of one image.  Returns false if the driver entry point is missing or
+// the encoder rejects the map.
 bool encode_region_map(CUtensorMap* map, const void* base, int B, int H, int W, int C, int box_w,
-                       int box_h);
+                       int box_h, int box_c);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
