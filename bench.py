@@ -42,9 +42,9 @@ FALLBACK_HBM_GBS = 6650.0
 # an ncu capture, keyed by the sha256 of the kernel sources it was taken on;
 # reported as ``traffic`` only while the sources are unchanged.
 TRAFFIC_RECORDS: dict[str, float] = {
-    # ncu --set full capture of bra_attend_stack_kernel<2, 1> on the stage-1 workload:
-    # dram__bytes_read.sum 68.27 MB + dram__bytes_write.sum 4.69 MB
-    "5462cc13d057e282ac9b4010070a844de12aed4c4fd6ac554cb4857872960366": 72.962048e6,
+    # ncu --set full capture of bra_attend_stack_kernel<4, 1> on the stage-1 workload:
+    # dram__bytes_read.sum 68.27 MB + dram__bytes_write.sum 3.59 MB
+    "4d7532c4bbd12985ea2b31e37bd88ef8418c1707a8cf29f2632ea5ccc978ac81": 71.858688e6,
 }
 
 
@@ -102,7 +102,7 @@ def kernel_sources_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dynamic_sparse_attention_bra_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("attend") or name in ("common.cuh", "kernels.h"):
+        if name.startswith(("attend", "tma_host")) or name in ("common.cuh", "kernels.h", "tc_ptx.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()
