@@ -21,6 +21,11 @@
 // window the same for all lanes of a warp.  No score outside a window is
 // ever read, and P is zero outside the windows (each P row only ever writes
 // its own window), so O_h = P_h V_h (M = 64, N = 32) needs no masking either.
+// With several regions per half and windows of 64 keys or more, P is kept
+// compact instead (each row holds only its own window) and P V runs as one
+// accumulator per region -- compact P times that region's V window, rows of
+// other regions computing values no one reads -- so P is Gq times smaller and
+// the dependent 16-key steps of one accumulator are kn / 16, not Gq * kn / 16.
 //
 // Roles (one CTA per SM, tiles strided by the grid):
 //   warps 0-1  producers, tiles alternating between them: read the tile's
@@ -58,6 +63,7 @@ constexpr uint32_t kSmemBudget = 227 * 1024;
 
 struct StackPlan {
     int Gq;                 // query regions per half
+    int cp;                 // 1: compact P (each row keeps only its kn-key window; Gq > 1, kn >= 64)
     int kn;                 // keys per query region
     int N;                  // keys per half = Gq * kn (MMA N of Q K^T)
     int hp;                 // 1: halves are a head pair (heads even), 0: region groups of one head
@@ -128,8 +134,9 @@ struct RowState {
 };
 
 
-// WGS softmax warp groups (1, 2 or 4); KN64: every window is exactly 64 keys.
-template <int WGS, bool KN64>
+// WGS softmax warp groups (1, 2 or 4); KN64: every window is exactly 64 keys;
+// CP: compact P with one P V accumulator per query region.
+template <int WGS, bool KN64, bool CP>
 __global__ void __launch_bounds__(32 * kCtrl + 128 * WGS, 1)
 bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                         const __grid_constant__ CUtensorMap tv, const int32_t* __restrict__ idx,
@@ -362,15 +369,36 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 ptx::tc_fence_after();
                 const uint32_t stage = sbase + (uint32_t)s * p.stage_bytes;
                 const uint32_t pbase = sbase + p.p_off + (uint32_t)pb * 2u * p.p_half;
-                for (int kk = 0; kk < p.N / 16; ++kk) {
+                if constexpr (CP) {
+                    // One accumulator per (half, region g) over g's kn-key window, the
+                    // O blocks 48 columns apart; steps of all accumulators interleaved.
+                    const int steps = p.kn / 16;
+                    for (int kk = 0; kk < steps; ++kk) {
+                        for (int gg = 0; gg < p.Gq; ++gg) {
+                            const int kg = gg * steps + kk;  // 16-key step of the half's stacked keys
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const uint32_t d = tmem + sbuf * p.N + ((uint32_t)(half * 16) << 16);
-                        const uint64_t a = ptx::smem_desc(pbase + half * p.p_half + (kk >> 2) * 8192 + (kk & 3) * 32,
-                                                          16, 1024, ptx::kSwizzle128B);
-                        const uint32_t vaddr = stage + p.v_off + (uint32_t)half * p.N * 64 + kk * 1024;
-                        const uint64_t bd = ptx::smem_desc(vaddr, ones + kk * 1024 - vaddr, 512, ptx::kSwizzle64B);
-                        ptx::mma_bf16(d, a, bd, idesc_pv, kk);
+                            for (int half = 0; half < 2; ++half) {
+                                const uint32_t d = tmem + sbuf * p.N + (uint32_t)gg * 48u + ((uint32_t)(half * 16) << 16);
+                                const uint64_t a = ptx::smem_desc(pbase + half * p.p_half + (kk >> 2) * 8192 + (kk & 3) * 32,
+                                                                  16, 1024, ptx::kSwizzle128B);
+                                const uint32_t vaddr = stage + p.v_off + (uint32_t)half * p.N * 64 + kg * 1024;
+                                const uint64_t bd = ptx::smem_desc(vaddr, ones + kg * 1024 - vaddr, 512, ptx::kSwizzle64B);
+                                ptx::mma_bf16(d, a, bd, idesc_pv, kk);
+                            }
+                        }
+                    }
+                } else {
+                    // Block-diagonal P: one accumulator per half over all N keys.
+                    for (int kk = 0; kk < p.N / 16; ++kk) {
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const uint32_t d = tmem + sbuf * p.N + ((uint32_t)(half * 16) << 16);
+                            const uint64_t a = ptx::smem_desc(pbase + half * p.p_half + (kk >> 2) * 8192 + (kk & 3) * 32,
+                                                              16, 1024, ptx::kSwizzle128B);
+                            const uint32_t vaddr = stage + p.v_off + (uint32_t)half * p.N * 64 + kk * 1024;
+                            const uint64_t bd = ptx::smem_desc(vaddr, ones + kk * 1024 - vaddr, 512, ptx::kSwizzle64B);
+                            ptx::mma_bf16(d, a, bd, idesc_pv, kk);
+                        }
                     }
                 }
                 ptx::mma_commit(&sb->o_full[sbuf]);
@@ -403,9 +431,10 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             // l (column 32) with O columns 0-15, then O columns 16-31: no more
             // than 17 accumulator words are held at a time.
             uint32_t r[16], lw = 0;
+            const uint32_t o_col = sbuf * p.N + (CP ? (uint32_t)slot * 48u : 0u);  // this row's O block
             if (slot_ok) {
-                ptx::tmem_ld16(tmem + lane_addr + sbuf * p.N, r);
-                lw = ptx::tmem_ld1(tmem + lane_addr + sbuf * p.N + 32);
+                ptx::tmem_ld16(tmem + lane_addr + o_col, r);
+                lw = ptx::tmem_ld1(tmem + lane_addr + o_col + 32);
                 ptx::tmem_wait17(r, lw);
             }
             const float l = __uint_as_float(lw);
@@ -416,7 +445,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
                 if (h16 == 1 && slot_ok) {
-                    ptx::tmem_ld16(tmem + lane_addr + sbuf * p.N + 16, r);
+                    ptx::tmem_ld16(tmem + lane_addr + o_col + 16, r);
                     ptx::tmem_wait16(r);
                 }
                 if (write) {
@@ -457,7 +486,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 // 16 p values of window columns c .. c + 15 as 8 bf16 pairs: two
                 // 16-byte chunks of the row's 128-byte swizzled atom line.
                 auto write_p16 = [&](int c, const uint32_t* packed) {
-                    const int col = slot * p.kn + c;  // window column inside the half's P
+                    const int col = CP ? c : slot * p.kn + c;  // column of the row's P
                     const uint32_t atom = prow + (uint32_t)(col >> 6) * 8192u;
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
@@ -575,7 +604,8 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     p->k_off = 8192;
     p->v_off = 8192 + kv;
     p->stage_bytes = 8192 + 2 * kv;
-    p->p_half = (uint32_t)((p->N + 63) / 64) * 8192u;
+    p->cp = (p->Gq > 1 && kn >= 64) ? 1 : 0;  // Gq O blocks of 48 columns fit in the N S columns
+    p->p_half = (uint32_t)(((p->cp ? kn : p->N) + 63) / 64) * 8192u;
     const uint32_t misc = (uint32_t)((sizeof(Barriers) + 1023) / 1024 * 1024);
     const uint32_t ones_bytes = (uint32_t)p->N * 64u;  // N keys x 64 B of bf16 ones
     if (512 / p->N < 2) return false;
@@ -585,10 +615,10 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     // on a barrier's parity need the barrier's previous phase complete: a
     // group's earlier tiles must cover the tile `stages` (and `nsb`) before,
     // so groups <= stages and nsb a multiple of the groups.
-    static const int kOptions[5][3] = {{4, 1, 5}, {2, 2, 3}, {2, 1, 3}, {1, 2, 3}, {1, 1, 2}};
+    static const int kOptions[6][3] = {{4, 1, 5}, {2, 2, 3}, {2, 1, 3}, {1, 2, 3}, {2, 1, 2}, {1, 1, 2}};
     int stages = 0;
     bool found = false;
-    for (int o = 0; o < 5 && !found; ++o) {
+    for (int o = 0; o < 6 && !found; ++o) {
         if (kOptions[o][0] > max_groups || p->nsb % kOptions[o][0] != 0) continue;
         p->wgs = kOptions[o][0];
         p->pdepth = kOptions[o][1];
@@ -631,9 +661,17 @@ bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, 
     const int sms = sm_count();
     if (sms <= 0) return BRA_ERR_CUDA;
     const int grid = p.tiles < sms ? p.tiles : sms;
-    auto kernel = p.wgs == 4   ? (p.kn == 64 ? bra_attend_stack_kernel<4, true> : bra_attend_stack_kernel<4, false>)
-                  : p.wgs == 2 ? (p.kn == 64 ? bra_attend_stack_kernel<2, true> : bra_attend_stack_kernel<2, false>)
-                               : (p.kn == 64 ? bra_attend_stack_kernel<1, true> : bra_attend_stack_kernel<1, false>);
+    using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, const int32_t*, __nv_bfloat16*, Geometry,
+                              StackPlan, int*);
+    // [cp][groups 1, 2, 4][kn == 64]
+    static const KernelFn kKernels[2][3][2] = {
+        {{bra_attend_stack_kernel<1, false, false>, bra_attend_stack_kernel<1, true, false>},
+         {bra_attend_stack_kernel<2, false, false>, bra_attend_stack_kernel<2, true, false>},
+         {bra_attend_stack_kernel<4, false, false>, bra_attend_stack_kernel<4, true, false>}},
+        {{bra_attend_stack_kernel<1, false, true>, bra_attend_stack_kernel<1, true, true>},
+         {bra_attend_stack_kernel<2, false, true>, bra_attend_stack_kernel<2, true, true>},
+         {bra_attend_stack_kernel<4, false, true>, bra_attend_stack_kernel<4, true, true>}}};
+    const KernelFn kernel = kKernels[p.cp][p.wgs == 4 ? 2 : p.wgs - 1][p.kn == 64 ? 1 : 0];
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes) !=
         cudaSuccess)
         return BRA_ERR_CUDA;
