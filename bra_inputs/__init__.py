@@ -152,6 +152,9 @@ WORKLOADS = {
     "stage2": (BraShape(64, 28, 28, 128, 4, 7, 4, "bf16"), 2),
     "stage3": (BraShape(64, 14, 14, 256, 8, 7, 16, "bf16"), 3),
     "highres": (BraShape(2, 128, 128, 64, 2, 8, 4, "bf16"), 4),
+    # object detection uses S = 16 (a 512 x 512 input at stride 4: 128 x 128 tokens,
+    # 256 regions of 8 x 8)
+    "detection": (BraShape(2, 128, 128, 64, 2, 16, 4, "bf16"), 5),
 }
 
 

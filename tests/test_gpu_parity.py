@@ -79,6 +79,16 @@ EXTRA = {
     "max_regions": (1, 32, 32, 32, 1, 16, 8, "bf16"),       # R = 256
     "many_heads": (1, 14, 14, 512, 16, 7, 16, "bf16"),
     "long_route_f32": (1, 32, 32, 32, 1, 4, 12, "f32"),     # 768 keys per query
+    # S / k ablation of the BiFormer pages (per-image geometry of each stage, batch 8):
+    # S = 7 with k = [1, 2, 8, 32] and S = [8, 4, 2, 1] with k = [2, 2, 2, 1]
+    "ablation_k2_stage2": (8, 28, 28, 128, 4, 7, 2, "bf16"),   # 32 keys per query
+    "ablation_k8_stage3": (8, 14, 14, 256, 8, 7, 8, "bf16"),   # 32 keys per query
+    "ablation_k32_stage4": (8, 7, 7, 512, 16, 7, 32, "bf16"),  # one-token regions
+    "stage4_full": (8, 7, 7, 512, 16, 7, 49, "bf16"),          # k = S^2: full attention
+    "ablation_s8_stage1": (8, 56, 56, 64, 2, 8, 2, "bf16"),    # 49-token regions, 98 keys
+    "ablation_s4_stage2": (8, 28, 28, 128, 4, 4, 2, "bf16"),
+    "ablation_s2_stage3": (8, 14, 14, 256, 8, 2, 2, "bf16"),
+    "ablation_s1_stage4": (8, 7, 7, 512, 16, 1, 1, "bf16"),    # one region: dense
 }
 
 
