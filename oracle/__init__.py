@@ -50,6 +50,7 @@ def _bind(path: str):
     lib.oracle_topk_routing.argtypes = [_dp, _i, _i, _i, _i, _ip]
     lib.oracle_token_attention.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _ip, _dp]
     lib.oracle_bra_forward.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _dp, _ip, _dp]
+    lib.oracle_local_context.argtypes = [_dp, _i, _i, _i, _i, _dp, _dp, _dp]
     for f in (lib.oracle_region_pool, lib.oracle_region_affinity, lib.oracle_topk_routing,
               lib.oracle_token_attention, lib.oracle_bra_forward):
         f.restype = _i
@@ -143,3 +144,19 @@ def bra_forward(q, k, v, heads: int, S: int, topk: int, want_affinity: bool = Fa
                                     _ptr(a, _dp) if a is not None else None)
     _check(rc, "forward")
     return (o, idx, a) if want_affinity else (o, idx)
+
+
+def local_context(v, weight, bias=None) -> np.ndarray:
+    """5x5 depthwise filter of V (zero padding 2, cross-correlation) plus bias:
+    the local context enhancement term added to the attention output.
+    ``weight`` is [C, 5, 5] (a [C, 1, 5, 5] layer weight reshaped), ``bias`` [C]
+    or None."""
+    v = _f64(v)
+    B, H, W, C = v.shape
+    w = _f64(np.reshape(weight, (C, 5, 5)))
+    bb = _f64(bias) if bias is not None else None
+    out = np.zeros_like(v)
+    _check(_load().oracle_local_context(_ptr(v, _dp), B, H, W, C, _ptr(w, _dp),
+                                        _ptr(bb, _dp) if bb is not None else None, _ptr(out, _dp)),
+           "local context")
+    return out

@@ -30,8 +30,12 @@
  *   - region order and token order inside a region are row-major;
  *   - top-k ties go to the lower region index, and each I^r row lists its
  *     regions by (affinity descending, index ascending);
- *   - the local-context term (5x5 depthwise convolution of V) is not part
- *     of this path.
+ *   - the local-context term (section 2.2 step 4, third bullet, and the
+ *     "+ dwconv(value)" of pseudocode step 7) is a separate function,
+ *     oracle_local_context: a 5x5 depthwise filter over the H x W map with
+ *     caller-given weights [C][5][5] and an optional bias [C] (the pages give
+ *     neither), stride 1, zero padding 2, applied as a cross-correlation
+ *     (the convention of deep-learning convolution layers).
  *
  * Layouts: Q, K, V, O are [B, H, W, C] channels-last float64; Q^r, K^r are
  * [B, heads, R, d]; A^r is [B, heads, R, R]; I^r is [B, heads, R, topk]
@@ -216,4 +220,33 @@ done:
     free(kr);
     if (!a) free(aa);
     return rc;
+}
+
+/* Local context enhancement (section 2.2 step 4, third bullet; pseudocode
+ * step 7 adds it to the attention output): for every channel c,
+ *   out[b, y, x, c] = bias[c] + sum_{i, j = 0..4} w[c][i][j] * v[b, y + i - 2, x + j - 2, c]
+ * with v = 0 outside the map.  ``bias`` may be NULL (no bias).  Plain loops,
+ * taps in (i, j) row-major order. */
+int oracle_local_context(const double* v, int B, int H, int W, int C, const double* w,
+                         const double* bias, double* out)
+{
+    if (B < 0 || H <= 0 || W <= 0 || C <= 0) return ORACLE_EINVAL;
+    for (int b = 0; b < B; ++b)
+        for (int y = 0; y < H; ++y)
+            for (int x = 0; x < W; ++x)
+                for (int c = 0; c < C; ++c) {
+                    double acc = bias ? bias[c] : 0.0;
+                    for (int i = 0; i < 5; ++i) {
+                        int yy = y + i - 2;
+                        if (yy < 0 || yy >= H) continue;
+                        for (int j = 0; j < 5; ++j) {
+                            int xx = x + j - 2;
+                            if (xx < 0 || xx >= W) continue;
+                            acc += w[(size_t)c * 25 + i * 5 + j] *
+                                   v[(((size_t)b * H + yy) * W + xx) * C + c];
+                        }
+                    }
+                    out[(((size_t)b * H + y) * W + x) * C + c] = acc;
+                }
+    return 0;
 }

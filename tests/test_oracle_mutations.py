@@ -61,3 +61,34 @@ def test_pins_catch_mutation(tmp_path, name, old, new):
             except (AssertionError, ValueError):
                 failures += 1
     assert failures > 0, f"no pin caught mutation {name}"
+
+
+# The local context term's pins catch slips in its own function.
+LCE_MUTATIONS = [
+    ("lce_convolution_orientation", "int yy = y + i - 2;", "int yy = y - i + 2;"),
+    ("lce_clamped_border", "if (yy < 0 || yy >= H) continue;",
+     "if (yy < 0) yy = 0; if (yy >= H) yy = H - 1;"),
+    ("lce_bias_dropped", "double acc = bias ? bias[c] : 0.0;", "double acc = 0.0;"),
+    ("lce_taps_transposed", "acc += w[(size_t)c * 25 + i * 5 + j] *", "acc += w[(size_t)c * 25 + j * 5 + i] *"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", LCE_MUTATIONS, ids=[m[0] for m in LCE_MUTATIONS])
+def test_local_context_pins_catch_mutation(tmp_path, name, old, new):
+    import test_oracle_lce as pins
+    lib = build_variant(tmp_path, name, old, new)
+    checks = [
+        pins.test_matches_scipy_correlate2d_per_channel,
+        pins.test_identity_kernel_returns_v,
+        lambda: pins.test_single_tap_is_a_shift_with_zero_fill(1, -1),
+        pins.test_constant_input_gives_kernel_sums,
+        pins.test_bias_only,
+    ]
+    failures = 0
+    with oracle.swapped_library(lib):
+        for check in checks:
+            try:
+                check()
+            except AssertionError:
+                failures += 1
+    assert failures > 0, f"no pin caught mutation {name}"
