@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--workload", default=WORKLOAD, choices=list(bi.WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--lce", action="store_true",
+                   help="add the local context enhancement (bra_lce, seeded 5x5 depthwise weights) to every step")
     return p.parse_args()
 
 
@@ -198,10 +200,18 @@ def run_reference(args):
     import oracle
     inp = bi.make_inputs(shape, seed)
     bpc = 1  # one image per step: a bounded sample of the batch
-    step = lambda i: oracle.bra_forward(inp.q_f64[i % shape.B:i % shape.B + bpc],
-                                        inp.k_f64[i % shape.B:i % shape.B + bpc],
-                                        inp.v_f64[i % shape.B:i % shape.B + bpc],
-                                        shape.heads, shape.S, shape.topk)
+    lce_w = lce_b = None
+    if args.lce:
+        rng = np.random.default_rng(seed + 77)
+        lce_w = rng.standard_normal((shape.C, 5, 5)) / 5.0
+        lce_b = rng.standard_normal(shape.C)
+
+    def step(i):
+        sl = slice(i % shape.B, i % shape.B + bpc)
+        o, _ = oracle.bra_forward(inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl], shape.heads, shape.S, shape.topk)
+        if args.lce:
+            o = o + oracle.local_context(inp.v_f64[sl], lce_w, lce_b)
+        return o
     for i in range(args.warmup):
         step(i)
     t0 = time.perf_counter()
@@ -215,7 +225,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**workload_config(shape, args.workload), "sample_images_per_step": bpc},
+        "config": {**workload_config(shape, args.workload), "sample_images_per_step": bpc,
+                   "local_context": bool(args.lce)},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"{bpc} of {shape.B} images per step, float64 oracle, one thread"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -260,9 +271,18 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=dev)
     sp = stream.cuda_stream
 
+    # local context enhancement parameters (seeded, as a layer's weights would be)
+    lce_w = lce_b = None
+    if args.lce:
+        g = torch.Generator().manual_seed(seed + 77)
+        lce_w = (torch.randn(shape.C * 25, generator=g) / 5.0).to(dev)
+        lce_b = torch.randn(shape.C, generator=g).to(dev)
+
     def step(i):
         b = sets[i % nsets]
         bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+        if args.lce:
+            bra.bra_lce(s, b["v"], lce_w, lce_b, b["o"], sp)
 
     for i in range(args.warmup):
         step(i)
@@ -319,6 +339,8 @@ def run_ours(args):
             for dst, src in zip((b0["q"], b0["k"], b0["v"]), host_qkv):
                 dst.copy_(src, non_blocking=True)
             bra.bra_forward(s, b0["q"], b0["k"], b0["v"], b0["o"], b0["idx"], b0["ws"], sp)
+            if args.lce:
+                bra.bra_lce(s, b0["v"], lce_w, lce_b, b0["o"], sp)
             o_host.copy_(b0["o"], non_blocking=True)
             idx_host.copy_(b0["idx"], non_blocking=True)
 
@@ -354,6 +376,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": shape.dtype, "data": "synthetic",
             "config": {**workload_config(shape, args.workload), "parallelism": f"replicas{world}",
+                       "local_context": bool(args.lce),
                        "l2": f"rotating {nsets} input sets ({nsets * set_bytes / 2**20:.0f} MiB) > 126 MiB L2"},
             "roofline": {
                 "kernel": "bra_attend", "bound": "hbm", "achieved": achieved, "peak": peak,
@@ -367,7 +390,7 @@ def run_ours(args):
             },
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (4 if args.lce else 3) * args.steps,
             "clocks": clocks.report(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -25,7 +25,7 @@ import os
 __all__ = [
     "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
     "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
-    "bra_route_noalloc",
+    "bra_route_noalloc", "bra_lce",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -36,7 +36,8 @@ BRA_OK, BRA_ERR_INVALID_ARG, BRA_ERR_UNSUPPORTED, BRA_ERR_CUDA, BRA_ERR_TIMEOUT,
 BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
-                    "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc")
+                    "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc",
+                    "bra_lce")
 NOALLOC_MAX_MEANS = 1 << 20  # BRA_NOALLOC_MAX_MEANS
 
 
@@ -56,7 +57,7 @@ class BraError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(library_path):
         raise ImportError(
-            f"{library_path} is not built; run `python -m dynamic_sparse_attention_bra_b200.build`")
+            f"{library_path} is not built; run `python dynamic_sparse_attention_bra_b200/build.py`")
     lib = ctypes.CDLL(library_path)
     vp, sp = ctypes.c_void_p, ctypes.POINTER(BraShape)
     lib.bra_workspace_bytes.argtypes = [sp]
@@ -64,6 +65,7 @@ def _load() -> ctypes.CDLL:
     lib.bra_route.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.bra_attend.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
+    lib.bra_lce.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.bra_device_status.argtypes = [sp, vp, vp]
     lib.bra_route_noalloc.argtypes = [sp, vp, vp, vp, vp]
     lib.bra_route_noalloc.restype = ctypes.c_int
@@ -123,6 +125,12 @@ def bra_attend(shape: BraShape, q, k, v, idx, o, workspace, stream=None) -> None
 def bra_forward(shape: BraShape, q, k, v, o, idx, workspace, stream=None) -> None:
     _check(_lib.bra_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(idx),
                             _ptr(workspace), _stream(stream)), "bra_forward")
+
+
+def bra_lce(shape: BraShape, v, weight, bias, o, stream=None) -> None:
+    """o += bias + 5x5 depthwise filter of v (weight fp32 [C, 5, 5], bias fp32 [C] or None)."""
+    _check(_lib.bra_lce(ctypes.byref(shape), _ptr(v), _ptr(weight), _ptr(bias) if bias is not None else None,
+                        _ptr(o), _stream(stream)), "bra_lce")
 
 
 def bra_route_noalloc(shape: BraShape, q, k, idx, stream=None) -> None:

@@ -1,7 +1,9 @@
 """Builds the sm_100a shared library ``libbra_b200.so`` in place with nvcc.
 
-Run as ``python -m dynamic_sparse_attention_bra_b200.build``; compiling
-needs nvcc only (no GPU).  Every ``csrc/*.cu`` file goes into one library.
+Run as ``python dynamic_sparse_attention_bra_b200/build.py`` (by path: the
+package itself loads the library on import, so it cannot be imported before
+the library exists); compiling needs nvcc only (no GPU).  Every ``csrc/*.cu``
+file goes into one library.
 """
 from __future__ import annotations
 

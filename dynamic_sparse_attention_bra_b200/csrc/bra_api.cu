@@ -166,6 +166,21 @@ bra_status bra_forward(const bra_shape* shape, const void* q, const void* k, con
     return attend_impl(shape, g, q, k, v, idx, o, w, st);
 }
 
+bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, const float* bias, void* o,
+                   void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!v || !weight || !o) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(v) || !aligned16(o) || !aligned16(weight) || (bias && !aligned16(bias)))
+        return BRA_ERR_INVALID_ARG;
+    if ((int64_t)g.H > (int64_t)65535 * 8) return BRA_ERR_UNSUPPORTED;  // grid rows of 8 outputs
+    return launch_lce(shape->dtype == BRA_DTYPE_BF16, v, weight, bias, o, g, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? BRA_OK
+               : BRA_ERR_CUDA;
+}
+
 bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stream) {
     Geometry g;
     bra_status rc = make_geometry(shape, &g);

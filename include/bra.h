@@ -127,6 +127,30 @@ bra_status bra_forward(const bra_shape* shape, const void* q, const void* k, con
                        void* o, int32_t* idx, void* workspace, void* stream);
 
 /*
+ * Local context enhancement, added in place to an attention output (blog
+ * "BiFormer Reshapes Visual Attention with Bi-Level Routing", Part 2 section
+ * 2.2, step 4 third bullet; pseudocode step 7 adds "dwconv(value)" to the
+ * attention result).  For every b, y, x and channel c:
+ *   o[b,y,x,c] += bias[c] + sum_{i,j=0..4} weight[c][i][j] * v[b, y+i-2, x+j-2, c]
+ * with v = 0 outside the H x W map: a 5x5 depthwise filter, stride 1, zero
+ * padding 2, in the cross-correlation orientation of deep-learning
+ * convolution layers.  The pages give no weights, bias or padding; the caller
+ * supplies the layer's parameters.  Accumulation is fp32; a bf16 ``o`` is
+ * read, the term added in fp32 and the sum rounded to nearest-even once.
+ *   shape      as for bra_forward (only B, H, W, C and dtype are used by the
+ *              filter; the other fields are checked as for bra_forward)
+ *   v          device, [B, H, W, C] of ``shape->dtype``, read only
+ *   weight     device fp32 [C][5][5] (a [C, 1, 5, 5] layer weight), read only
+ *   bias       device fp32 [C], or NULL for no bias
+ *   o          device, [B, H, W, C] of ``shape->dtype``, read and written
+ * All pointers 16-byte aligned.  Errors: as bra_route (BRA_ERR_INVALID_ARG
+ * for a bad shape or a null/misaligned pointer, before any launch;
+ * BRA_ERR_CUDA if the launch fails).  Runs on ``stream``; allocates nothing.
+ */
+bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, const float* bias, void* o,
+                   void* stream);
+
+/*
  * Reads (synchronising ``stream``) and clears the device status block in
  * ``workspace``: BRA_OK, BRA_ERR_TIMEOUT (a bounded wait in a kernel gave up;
  * that kernel's outputs are incomplete) or BRA_ERR_BAD_ROUTE.

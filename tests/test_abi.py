@@ -76,6 +76,7 @@ def test_bad_shapes_rejected_before_launch(bad, code):
     assert bra._lib.bra_forward(ctypes.byref(s), p, p, p, p, p, p, None) == code
     assert bra._lib.bra_route(ctypes.byref(s), p, p, p, p, None) == code
     assert bra._lib.bra_attend(ctypes.byref(s), p, p, p, p, p, p, None) == code
+    assert bra._lib.bra_lce(ctypes.byref(s), p, p, p, p, None) == code
     assert bra.bra_workspace_bytes(s) == 0
 
 
@@ -109,3 +110,16 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+@pytest.mark.parametrize("which", range(4))
+def test_lce_null_and_misaligned_pointers(which):
+    """v, weight, o must be non-null and 16-byte aligned; bias may be null but
+    not misaligned.  Every case is rejected on the host, before any launch."""
+    s = shp()
+    good = [1 << 20] * 4
+    for bad in ((0, (1 << 20) + 4) if which != 2 else ((1 << 20) + 4,)):
+        ptrs = list(good)
+        ptrs[which] = bad
+        v, w, b, o = ptrs
+        assert bra._lib.bra_lce(ctypes.byref(s), v, w, b, o, None) == bra.BRA_ERR_INVALID_ARG
