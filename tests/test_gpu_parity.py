@@ -89,6 +89,7 @@ EXTRA = {
     "ablation_s4_stage2": (8, 28, 28, 128, 4, 4, 2, "bf16"),
     "ablation_s2_stage3": (8, 14, 14, 256, 8, 2, 2, "bf16"),
     "ablation_s1_stage4": (8, 7, 7, 512, 16, 1, 1, "bf16"),    # one region: dense
+    "three_heads": (4, 28, 28, 96, 3, 7, 4, "bf16"),           # 12 vectors per token: region-form pooling
 }
 
 
@@ -230,3 +231,31 @@ def test_stack_kernel_groups(groups, name, monkeypatch):
         B, H, W, C, heads, S, topk, dtype = EXTRA[name]
         shape, seed = bi.BraShape(B, H, W, C, heads, S, topk, dtype), 11
     check_case(shape, seed)
+
+
+def test_workspace_reused_across_calls():
+    """One workspace serves any number of ordered calls: each call on a reused
+    workspace gives bit-identical results to the same call on a fresh one."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    from gpu_helpers import device_inputs
+    shape, _ = bi.WORKLOADS["stage2"]
+    sh = bi.BraShape(8, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    s = bra.shape_for(sh.B, sh.H, sh.W, sh.C, sh.heads, sh.S, sh.topk, sh.dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    for seed in (21, 22, 23):
+        inp = bi.make_inputs(sh, seed)
+        q, k, v = device_inputs(inp)
+        o = torch.empty_like(q)
+        idx = torch.empty((sh.B, sh.heads, sh.R, sh.topk), dtype=torch.int32, device="cuda")
+        bra.bra_forward(s, q, k, v, o, idx, ws)
+        assert bra.bra_device_status(s, ws) == bra.BRA_OK
+        torch.cuda.synchronize()
+        # the same call on a fresh workspace gives bit-identical results
+        ws2 = torch.zeros_like(ws)
+        o2 = torch.empty_like(q)
+        idx2 = torch.empty_like(idx)
+        bra.bra_forward(s, q, k, v, o2, idx2, ws2)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, idx2)
+        assert torch.equal(o.view(torch.int16), o2.view(torch.int16))
