@@ -25,7 +25,7 @@ import os
 __all__ = [
     "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
     "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
-    "bra_route_noalloc", "bra_lce",
+    "bra_route_noalloc", "bra_lce", "bra_selftest_bounded_wait",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -37,7 +37,7 @@ BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
                     "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc",
-                    "bra_lce")
+                    "bra_lce", "bra_selftest_bounded_wait")
 NOALLOC_MAX_MEANS = 1 << 20  # BRA_NOALLOC_MAX_MEANS
 
 
@@ -66,6 +66,7 @@ def _load() -> ctypes.CDLL:
     lib.bra_attend.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_lce.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.bra_selftest_bounded_wait.argtypes = [sp, vp, ctypes.c_uint, ctypes.c_int, vp]
     lib.bra_device_status.argtypes = [sp, vp, vp]
     lib.bra_route_noalloc.argtypes = [sp, vp, vp, vp, vp]
     lib.bra_route_noalloc.restype = ctypes.c_int
@@ -125,6 +126,13 @@ def bra_attend(shape: BraShape, q, k, v, idx, o, workspace, stream=None) -> None
 def bra_forward(shape: BraShape, q, k, v, o, idx, workspace, stream=None) -> None:
     _check(_lib.bra_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(idx),
                             _ptr(workspace), _stream(stream)), "bra_forward")
+
+
+def bra_selftest_bounded_wait(shape: BraShape, workspace, tries: int, arrive: bool, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see include/bra.h); read the
+    outcome with bra_device_status."""
+    _check(_lib.bra_selftest_bounded_wait(ctypes.byref(shape), _ptr(workspace), tries, 1 if arrive else 0,
+                                          _stream(stream)), "bra_selftest_bounded_wait")
 
 
 def bra_lce(shape: BraShape, v, weight, bias, o, stream=None) -> None:

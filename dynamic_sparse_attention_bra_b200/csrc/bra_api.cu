@@ -181,6 +181,18 @@ bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, c
                : BRA_ERR_CUDA;
 }
 
+bra_status bra_selftest_bounded_wait(const bra_shape* shape, void* workspace, unsigned int tries, int arrive,
+                                     void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!workspace || !aligned16(workspace) || tries == 0 || tries > (1u << 24)) return BRA_ERR_INVALID_ARG;
+    return launch_bounded_wait_selftest(carve(g, workspace).status, tries, arrive != 0,
+                                        static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? BRA_OK
+               : BRA_ERR_CUDA;
+}
+
 bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stream) {
     Geometry g;
     bra_status rc = make_geometry(shape, &g);

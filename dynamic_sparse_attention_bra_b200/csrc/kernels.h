@@ -18,6 +18,9 @@ cudaError_t launch_pool(bool bf16, const void* q, const void* k, float* qr, floa
                         const Geometry& g, cudaStream_t stream);
 cudaError_t launch_route(const float* qr, const float* kr, int32_t* idx, const Geometry& g,
                          cudaStream_t stream);
+// Bounded-wait self-test: waits on an mbarrier nobody arrives at (unless
+// ``arrive``) for at most ``tries`` polls, then records kDevTimeout.
+cudaError_t launch_bounded_wait_selftest(int* status, uint32_t tries, bool arrive, cudaStream_t stream);
 // Local context enhancement: o += bias + 5x5 depthwise filter of v.
 cudaError_t launch_lce(bool bf16, const void* v, const float* w, const float* bias, void* o, const Geometry& g,
                        cudaStream_t stream);

@@ -178,6 +178,21 @@ bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stre
 bra_status bra_route_noalloc(const bra_shape* shape, const void* q, const void* k, int32_t* idx,
                              void* stream);
 
+/*
+ * Self-test of the failure-detection path (the pages have no counterpart):
+ * every kernel that waits on an mbarrier polls it a bounded number of times
+ * and, when the limit runs out, records BRA_ERR_TIMEOUT in the workspace
+ * status block and returns instead of hanging.  This call launches one small
+ * kernel that waits, with a limit of ``tries`` polls (1 .. 2^24), on an
+ * mbarrier that nothing arrives at (``arrive`` = 0; the wait runs out and
+ * BRA_ERR_TIMEOUT is recorded) or that it arrives at itself first (``arrive``
+ * != 0; the wait succeeds and nothing is recorded).  Read the outcome with
+ * bra_device_status.  ``shape`` and ``workspace`` as for bra_route.  Errors:
+ * BRA_ERR_INVALID_ARG (bad shape, workspace or ``tries``), BRA_ERR_CUDA.
+ */
+bra_status bra_selftest_bounded_wait(const bra_shape* shape, void* workspace, unsigned int tries, int arrive,
+                                     void* stream);
+
 /* Static English text for a status code. */
 const char* bra_status_string(bra_status status);
 

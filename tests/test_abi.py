@@ -123,3 +123,12 @@ def test_lce_null_and_misaligned_pointers(which):
         ptrs[which] = bad
         v, w, b, o = ptrs
         assert bra._lib.bra_lce(ctypes.byref(s), v, w, b, o, None) == bra.BRA_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_arguments_before_launch():
+    s = shp()
+    ws = 1 << 20
+    assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), ws, 0, 0, None) == bra.BRA_ERR_INVALID_ARG
+    assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), ws, (1 << 24) + 1, 0, None) == bra.BRA_ERR_INVALID_ARG
+    assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), None, 10, 0, None) == bra.BRA_ERR_INVALID_ARG
+    assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), ws + 8, 10, 0, None) == bra.BRA_ERR_INVALID_ARG
