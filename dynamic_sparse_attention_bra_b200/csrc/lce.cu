@@ -33,6 +33,26 @@ constexpr int kLceThreads = 256;           // 8 warps x 4 strips = 32 columns
 constexpr int kHaloRows = kLceRows + 4, kHaloCols = kLceCols + 4;
 constexpr int kHaloChunks = kHaloRows * kHaloCols * 8;  // 16-byte chunks of the halo tile
 
+// Two fp32 lanes in one 64-bit register (x in the low half): sm_100a
+// multiplies and adds both with one fma.rn.f32x2, rounding each as fmaf would.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// bf16 pair -> packed fp32 pair (each bf16 is the high half of its float)
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t r) {
+    return f2_pack(__uint_as_float(r << 16), __uint_as_float(r & 0xffff0000u));
+}
+
 template <typename T>
 struct LceVec;  // the channels of one lane: 2 bf16 or 1 float
 template <>
@@ -101,6 +121,7 @@ bra_lce_kernel(const T* __restrict__ v, const float* __restrict__ w, const float
     ptx::cp_async_commit();
     int wgrp = -1;  // channel group whose taps are in registers
     float wt[CH][25], b0[CH];
+    uint64_t wt2[25], b2 = 0;  // the bf16 path keeps its two channels' taps packed
     for (int i = 0; t < tl.count; ++i, t += gridDim.x) {
         // the next tile streams into the other buffer while this one is computed
         if (t + (int)gridDim.x < tl.count) stage(t + gridDim.x, (i + 1) & 1);
@@ -111,6 +132,54 @@ bra_lce_kernel(const T* __restrict__ v, const float* __restrict__ w, const float
         coords(t, b, y0, x0, grp);
         const int c0 = grp * (128 / (int)sizeof(T)) + lane * CH;  // this lane's first channel
         if (c0 < C) {
+            const Raw* tile = reinterpret_cast<const Raw*>(lce_raw + (size_t)(i & 1) * kHaloChunks);  // 32 Raw per token
+            if constexpr (CH == 2) {
+                // bf16: the lane's two channels ride together in packed fp32 pairs
+                if (grp != wgrp) {
+#pragma unroll
+                    for (int tp = 0; tp < 25; ++tp)
+                        wt2[tp] = f2_pack(__ldg(w + (size_t)c0 * 25 + tp), __ldg(w + (size_t)(c0 + 1) * 25 + tp));
+                    b2 = bias ? f2_pack(__ldg(bias + c0), __ldg(bias + c0 + 1)) : f2_pack(0.f, 0.f);
+                    wgrp = grp;
+                }
+                for (int st = 0; st < kLceStrips; ++st) {
+                    const int cx = warp * kLceStrips + st;  // column inside the tile
+                    const int x = x0 + cx;
+                    if (x >= W) break;
+                    T* ob = o + ((size_t)b * H * W + (size_t)x) * C + c0;
+                    Raw cur_raw[kLceRows];
+#pragma unroll
+                    for (int r = 0; r < kLceRows; ++r)
+                        cur_raw[r] = y0 + r < H ? *reinterpret_cast<const Raw*>(ob + (size_t)(y0 + r) * W * C) : Raw(0);
+                    uint64_t acc[kLceRows];
+#pragma unroll
+                    for (int r = 0; r < kLceRows; ++r) acc[r] = b2;
+                    const Raw* colp = tile + cx * 32 + lane;
+#pragma unroll
+                    for (int k = 0; k < kHaloRows; ++k) {
+                        uint64_t f[5];
+#pragma unroll
+                        for (int j = 0; j < 5; ++j) f[j] = f2_from_bf16x2(colp[(k * kHaloCols + j) * 32]);
+#pragma unroll
+                        for (int r = 0; r < kLceRows; ++r) {
+                            const int ti = k - r;
+                            if (ti < 0 || ti > 4) continue;
+#pragma unroll
+                            for (int j = 0; j < 5; ++j) acc[r] = f2_fma(wt2[ti * 5 + j], f[j], acc[r]);
+                        }
+                    }
+#pragma unroll
+                    for (int r = 0; r < kLceRows; ++r) {
+                        if (y0 + r >= H) break;
+                        float cur[2], sum[2];
+                        V::unpack(cur_raw[r], cur);
+                        f2_unpack(acc[r], sum[0], sum[1]);
+                        sum[0] += cur[0];
+                        sum[1] += cur[1];
+                        *reinterpret_cast<Raw*>(ob + (size_t)(y0 + r) * W * C) = V::pack(sum);
+                    }
+                }
+            } else {
             if (grp != wgrp) {
 #pragma unroll
                 for (int e = 0; e < CH; ++e) {
@@ -120,7 +189,6 @@ bra_lce_kernel(const T* __restrict__ v, const float* __restrict__ w, const float
                 }
                 wgrp = grp;
             }
-            const Raw* tile = reinterpret_cast<const Raw*>(lce_raw + (size_t)(i & 1) * kHaloChunks);  // 32 Raw per token
             for (int st = 0; st < kLceStrips; ++st) {
                 const int cx = warp * kLceStrips + st;  // column inside the tile
                 const int x = x0 + cx;
@@ -164,6 +232,7 @@ bra_lce_kernel(const T* __restrict__ v, const float* __restrict__ w, const float
                 }
             }
         }
+            }
         __syncthreads();  // the buffer is free for the tile after next
     }
     ptx::cp_async_wait_all();
