@@ -48,7 +48,7 @@ TRAFFIC_RECORDS: dict[str, float] = {
 }
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=500)
@@ -59,7 +59,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--lce", action="store_true",
                    help="add the local context enhancement (bra_lce, seeded 5x5 depthwise weights) to every step")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 def workload_config(shape: bi.BraShape, name: str) -> dict:
@@ -185,6 +185,27 @@ def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
                       f"in {el:.1f} s, float64, one thread"}
 
 
+def max_over_ranks(values, world: int, device="cpu") -> list[float]:
+    """Element-wise maximum of ``values`` over all ranks (every rank gets it):
+    a multi-GPU time is the slowest rank's.  One process: ``values`` itself."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """All ranks' tokens of one step over the (slowest rank's) step time."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each replica draws its own batch."""
+    return seed + 1000 * rank
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -248,7 +269,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     shape, seed = bi.WORKLOADS[args.workload]
-    inp = bi.make_inputs(shape, seed + 1000 * rank)
+    inp = bi.make_inputs(shape, rank_seed(seed, rank))
     es = 2 if shape.dtype == "bf16" else 4
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
 
@@ -357,13 +378,10 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
 
-    times = torch.tensor([total_ms, attend_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    total_ms, attend_ms, e2e_ms = times.tolist()
+    total_ms, attend_ms, e2e_ms = max_over_ranks([total_ms, attend_ms, e2e_ms], world, dev)
     ms_per_step = total_ms / args.steps
     tokens = shape.tokens * world
-    value = tokens / (ms_per_step * 1e-3)
+    value = whole_job_tokens_per_s(shape.tokens, world, ms_per_step)
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
