@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 # reported as ``traffic`` only while the sources are unchanged.
 TRAFFIC_RECORDS: dict[str, float] = {
     # ncu --set full capture of bra_attend_stack_kernel<4, 1, 0> on the stage-1 workload:
-    # dram__bytes_read.sum 68.27 MB + dram__bytes_write.sum 3.96 MB
-    "5f40e01735b61958176475662da85c2b55498962dc87d974b32685519d73917f": 72.230144e6,
+    # dram__bytes_read.sum 68.28 MB + dram__bytes_write.sum 4.28 MB
+    "87a9b4f22773ee876f8e80b8c22ff2de3a6ec63af952d6ca7be72c780640a920": 72.554752e6,
 }
 
 

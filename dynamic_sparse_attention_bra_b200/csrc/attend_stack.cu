@@ -172,10 +172,20 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
         ptx::tmem_relinquish();
         ptx::tc_fence_before();
     }
-    // Zero every operand buffer once: stale rows outside a tile's loaded boxes
-    // are then always finite, and P stays zero outside each row's window.
-    for (uint32_t i = threadIdx.x; i < p.ones_off / 16; i += kThreads)
-        reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+    // Zero, once, what must not hold stale bits: the V rows of every stage (a
+    // dead route's P entries are zero, and 0 times a stale non-finite value
+    // would not be) and, when P is block-diagonal, the P buffers (zero outside
+    // each row's window).  Stale Q or K rows only reach scores no row reads.
+    {
+        const uint32_t v_chunks = (p.stage_bytes - p.v_off) / 16;
+        for (uint32_t i = threadIdx.x; i < (uint32_t)p.stages * v_chunks; i += kThreads) {
+            const uint32_t st = i / v_chunks, c = i - st * v_chunks;
+            reinterpret_cast<uint4*>(smem + st * p.stage_bytes + p.v_off)[c] = make_uint4(0, 0, 0, 0);
+        }
+        if (!CP && p.Gq > 1)
+            for (uint32_t i = p.p_off / 16 + threadIdx.x; i < p.ones_off / 16; i += kThreads)
+                reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+    }
     // A tile of bf16 ones (same shape as one V half): P times it gives every
     // row's sum of P on the tensor core.
     for (uint32_t i = p.ones_off / 16 + threadIdx.x; i < p.bar_off / 16; i += kThreads)
