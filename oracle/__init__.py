@@ -51,6 +51,7 @@ def _bind(path: str):
     lib.oracle_token_attention.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _ip, _dp]
     lib.oracle_bra_forward.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _dp, _ip, _dp]
     lib.oracle_local_context.argtypes = [_dp, _i, _i, _i, _i, _dp, _dp, _dp]
+    lib.oracle_attention_backward.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _ip, _dp, _dp, _dp, _dp]
     for f in (lib.oracle_region_pool, lib.oracle_region_affinity, lib.oracle_topk_routing,
               lib.oracle_token_attention, lib.oracle_bra_forward):
         f.restype = _i
@@ -160,3 +161,19 @@ def local_context(v, weight, bias=None) -> np.ndarray:
                                         _ptr(bb, _dp) if bb is not None else None, _ptr(out, _dp)),
            "local context")
     return out
+
+
+def attention_backward(q, k, v, idx, grad_o, heads: int, S: int):
+    """Gradients (dQ, dK, dV) of the token attention for a fixed routing
+    ``idx`` and an incoming gradient ``grad_o`` of O; a region repeated in a
+    routing row counts once."""
+    q, k, v, gr = _f64(q), _f64(k), _f64(v), _f64(grad_o)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    B, H, W, C = q.shape
+    topk = idx.shape[-1]
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    _check(_load().oracle_attention_backward(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), B, H, W, C, heads, S, topk,
+                                             _ptr(idx, _ip), _ptr(gr, _dp), _ptr(dq, _dp), _ptr(dk, _dp),
+                                             _ptr(dv, _dp)),
+           "attention backward")
+    return dq, dk, dv

@@ -250,3 +250,87 @@ int oracle_local_context(const double* v, int B, int H, int W, int C, const doub
                 }
     return 0;
 }
+
+/* Gradients of the token attention for a fixed routing (the backward of the
+ * step in section 2.2 step 4; top-k has no gradient, so I^r is an input).
+ * With s_j = <q_t, k_j> / sqrt(d), P = softmax(s), o_t = sum_j P_j v_j and an
+ * incoming gradient g_t = dL/do_t, the chain rule gives
+ *   dP_j = <g_t, v_j>,  D = sum_j P_j dP_j,  dS_j = P_j (dP_j - D),
+ *   dq_t += sum_j dS_j k_j / sqrt(d),  dk_j += dS_j q_t / sqrt(d),  dv_j += P_j g_t.
+ * The keys of a query are the tokens of its routed regions, a region listed
+ * twice counted once (first listing), as the library's attention does.
+ * dq, dk, dv are [B, H, W, C] float64, overwritten. */
+int oracle_attention_backward(const double* q, const double* k, const double* v,
+                              int B, int H, int W, int C, int heads, int S, int topk,
+                              const int32_t* idx, const double* g,
+                              double* dq, double* dk, double* dv)
+{
+    if (check_shape(B, H, W, C, heads, S, topk)) return ORACLE_EINVAL;
+    int R = S * S, d = C / heads, n = (H / S) * (W / S), kn = topk * n;
+    double scale = 1.0 / sqrt((double)d);
+    size_t total = (size_t)B * H * W * C;
+    memset(dq, 0, sizeof(double) * total);
+    memset(dk, 0, sizeof(double) * total);
+    memset(dv, 0, sizeof(double) * total);
+    double* p = (double*)malloc(sizeof(double) * (size_t)kn);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)kn);
+    size_t* key_off = (size_t*)malloc(sizeof(size_t) * (size_t)kn);
+    if (!p || !dp || !key_off) { free(p); free(dp); free(key_off); return ORACLE_ENOMEM; }
+    int rc = 0;
+    for (int b = 0; b < B && !rc; ++b)
+        for (int h = 0; h < heads && !rc; ++h)
+            for (int r = 0; r < R && !rc; ++r) {
+                const int32_t* route = idx + (((size_t)b * heads + h) * R + r) * topk;
+                int nk = 0;  /* keys of the distinct routed regions */
+                for (int m = 0; m < topk; ++m) {
+                    int rr = route[m];
+                    if (rr < 0 || rr >= R) { rc = ORACLE_EINVAL; break; }
+                    int seen = 0;
+                    for (int mm = 0; mm < m; ++mm) seen |= route[mm] == rr;
+                    if (seen) continue;
+                    for (int t = 0; t < n; ++t) {
+                        int y, x;
+                        region_token(H, W, S, rr, t, &y, &x);
+                        key_off[nk++] = (((size_t)b * H + y) * W + x) * C + (size_t)h * d;
+                    }
+                }
+                if (rc) break;
+                for (int t = 0; t < n; ++t) {
+                    int y, x;
+                    region_token(H, W, S, r, t, &y, &x);
+                    size_t qoff = (((size_t)b * H + y) * W + x) * C + (size_t)h * d;
+                    double mx = -INFINITY;
+                    for (int j = 0; j < nk; ++j) {
+                        double dot = 0.0;
+                        for (int c = 0; c < d; ++c) dot += q[qoff + c] * k[key_off[j] + c];
+                        p[j] = dot * scale;
+                        if (p[j] > mx) mx = p[j];
+                    }
+                    double den = 0.0;
+                    for (int j = 0; j < nk; ++j) {
+                        p[j] = exp(p[j] - mx);
+                        den += p[j];
+                    }
+                    double dsum = 0.0;
+                    for (int j = 0; j < nk; ++j) {
+                        p[j] /= den;
+                        double dot = 0.0;
+                        for (int c = 0; c < d; ++c) dot += g[qoff + c] * v[key_off[j] + c];
+                        dp[j] = dot;
+                        dsum += p[j] * dot;
+                    }
+                    for (int j = 0; j < nk; ++j) {
+                        double ds = p[j] * (dp[j] - dsum);
+                        for (int c = 0; c < d; ++c) {
+                            dq[qoff + c] += ds * k[key_off[j] + c] * scale;
+                            dk[key_off[j] + c] += ds * q[qoff + c] * scale;
+                            dv[key_off[j] + c] += p[j] * g[qoff + c];
+                        }
+                    }
+                }
+            }
+    free(p);
+    free(dp);
+    free(key_off);
+    return rc;
+}

@@ -92,3 +92,31 @@ def test_local_context_pins_catch_mutation(tmp_path, name, old, new):
             except AssertionError:
                 failures += 1
     assert failures > 0, f"no pin caught mutation {name}"
+
+
+# The attention-gradient pins catch slips in the backward function.
+BACKWARD_MUTATIONS = [
+    ("bwd_missing_mean_term", "double ds = p[j] * (dp[j] - dsum);", "double ds = p[j] * dp[j];"),
+    ("bwd_dk_unscaled", "dk[key_off[j] + c] += ds * q[qoff + c] * scale;", "dk[key_off[j] + c] += ds * q[qoff + c];"),
+    ("bwd_dv_from_ds", "dv[key_off[j] + c] += p[j] * g[qoff + c];", "dv[key_off[j] + c] += ds * g[qoff + c];"),
+    ("bwd_repeats_counted_twice", "                    if (seen) continue;\n", ""),
+]
+
+
+@pytest.mark.parametrize("name,old,new", BACKWARD_MUTATIONS, ids=[m[0] for m in BACKWARD_MUTATIONS])
+def test_backward_pins_catch_mutation(tmp_path, name, old, new):
+    import test_oracle_backward as pins
+    lib = build_variant(tmp_path, name, old, new)
+    checks = [
+        lambda: pins.test_gradients_match_finite_differences(1, 4, 4, 4, 1, 2, 2),
+        pins.test_full_routing_is_dense_attention_gradient,
+        pins.test_repeated_routes_count_once_like_a_masked_dense_attention,
+    ]
+    failures = 0
+    with oracle.swapped_library(lib):
+        for check in checks:
+            try:
+                check()
+            except AssertionError:
+                failures += 1
+    assert failures > 0, f"no pin caught mutation {name}"
