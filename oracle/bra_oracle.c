@@ -267,7 +267,7 @@ int oracle_attention_backward(const double* q, const double* k, const double* v,
 {
     if (check_shape(B, H, W, C, heads, S, topk)) return ORACLE_EINVAL;
     int R = S * S, d = C / heads, n = (H / S) * (W / S), kn = topk * n;
-    double scale = 1.0 / sqrt((double)d);
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);  /* the forward's logit scale */
     size_t total = (size_t)B * H * W * C;
     memset(dq, 0, sizeof(double) * total);
     memset(dk, 0, sizeof(double) * total);
@@ -283,14 +283,14 @@ int oracle_attention_backward(const double* q, const double* k, const double* v,
                 const int32_t* route = idx + (((size_t)b * heads + h) * R + r) * topk;
                 int nk = 0;  /* keys of the distinct routed regions */
                 for (int m = 0; m < topk; ++m) {
-                    int rr = route[m];
-                    if (rr < 0 || rr >= R) { rc = ORACLE_EINVAL; break; }
+                    int region = route[m];
+                    if (region < 0 || region >= R) { rc = ORACLE_EINVAL; break; }
                     int seen = 0;
-                    for (int mm = 0; mm < m; ++mm) seen |= route[mm] == rr;
+                    for (int mm = 0; mm < m; ++mm) seen |= route[mm] == region;
                     if (seen) continue;
                     for (int t = 0; t < n; ++t) {
                         int y, x;
-                        region_token(H, W, S, rr, t, &y, &x);
+                        region_token(H, W, S, region, t, &y, &x);
                         key_off[nk++] = (((size_t)b * H + y) * W + x) * C + (size_t)h * d;
                     }
                 }
@@ -303,7 +303,7 @@ int oracle_attention_backward(const double* q, const double* k, const double* v,
                     for (int j = 0; j < nk; ++j) {
                         double dot = 0.0;
                         for (int c = 0; c < d; ++c) dot += q[qoff + c] * k[key_off[j] + c];
-                        p[j] = dot * scale;
+                        p[j] = dot * inv_sqrt_d;
                         if (p[j] > mx) mx = p[j];
                     }
                     double den = 0.0;
@@ -322,8 +322,8 @@ int oracle_attention_backward(const double* q, const double* k, const double* v,
                     for (int j = 0; j < nk; ++j) {
                         double ds = p[j] * (dp[j] - dsum);
                         for (int c = 0; c < d; ++c) {
-                            dq[qoff + c] += ds * k[key_off[j] + c] * scale;
-                            dk[key_off[j] + c] += ds * q[qoff + c] * scale;
+                            dq[qoff + c] += ds * k[key_off[j] + c] * inv_sqrt_d;
+                            dk[key_off[j] + c] += ds * q[qoff + c] * inv_sqrt_d;
                             dv[key_off[j] + c] += p[j] * g[qoff + c];
                         }
                     }

@@ -97,7 +97,7 @@ def test_local_context_pins_catch_mutation(tmp_path, name, old, new):
 # The attention-gradient pins catch slips in the backward function.
 BACKWARD_MUTATIONS = [
     ("bwd_missing_mean_term", "double ds = p[j] * (dp[j] - dsum);", "double ds = p[j] * dp[j];"),
-    ("bwd_dk_unscaled", "dk[key_off[j] + c] += ds * q[qoff + c] * scale;", "dk[key_off[j] + c] += ds * q[qoff + c];"),
+    ("bwd_dk_unscaled", "dk[key_off[j] + c] += ds * q[qoff + c] * inv_sqrt_d;", "dk[key_off[j] + c] += ds * q[qoff + c];"),
     ("bwd_dv_from_ds", "dv[key_off[j] + c] += p[j] * g[qoff + c];", "dv[key_off[j] + c] += ds * g[qoff + c];"),
     ("bwd_repeats_counted_twice", "                    if (seen) continue;\n", ""),
 ]
