@@ -25,7 +25,7 @@ import os
 __all__ = [
     "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
     "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
-    "bra_route_noalloc", "bra_lce", "bra_selftest_bounded_wait",
+    "bra_route_noalloc", "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -37,7 +37,7 @@ BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
                     "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc",
-                    "bra_lce", "bra_selftest_bounded_wait")
+                    "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward")
 NOALLOC_MAX_MEANS = 1 << 20  # BRA_NOALLOC_MAX_MEANS
 
 
@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
     lib.bra_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_lce.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.bra_selftest_bounded_wait.argtypes = [sp, vp, ctypes.c_uint, ctypes.c_int, vp]
+    lib.bra_attend_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_device_status.argtypes = [sp, vp, vp]
     lib.bra_route_noalloc.argtypes = [sp, vp, vp, vp, vp]
     lib.bra_route_noalloc.restype = ctypes.c_int
@@ -126,6 +127,13 @@ def bra_attend(shape: BraShape, q, k, v, idx, o, workspace, stream=None) -> None
 def bra_forward(shape: BraShape, q, k, v, o, idx, workspace, stream=None) -> None:
     _check(_lib.bra_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(idx),
                             _ptr(workspace), _stream(stream)), "bra_forward")
+
+
+def bra_attend_backward(shape: BraShape, q, k, v, idx, grad_o, dq, dk, dv, workspace, stream=None) -> None:
+    """dQ, dK, dV (fp32 tensors, overwritten) of bra_attend for the fixed routing ``idx``."""
+    _check(_lib.bra_attend_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(grad_o),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream)),
+           "bra_attend_backward")
 
 
 def bra_selftest_bounded_wait(shape: BraShape, workspace, tries: int, arrive: bool, stream=None) -> None:

@@ -8,6 +8,7 @@
 
 #include "../../include/bra.h"
 #include "attend_tc.h"
+#include "backward.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -177,6 +178,30 @@ bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, c
     if ((int64_t)g.H > (int64_t)65535 * 8) return BRA_ERR_UNSUPPORTED;  // grid rows of 8 outputs
     return launch_lce(shape->dtype == BRA_DTYPE_BF16, v, weight, bias, o, g, static_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
+               ? BRA_OK
+               : BRA_ERR_CUDA;
+}
+
+bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const void* grad_o, float* dq, float* dk, float* dv,
+                               void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!q || !k || !v || !idx || !grad_o || !dq || !dk || !dv || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(grad_o) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    if (backward_smem_bytes(g) == 0) return BRA_ERR_UNSUPPORTED;
+    if ((long long)g.B * g.heads > 65535) return BRA_ERR_UNSUPPORTED;  // one grid row per (batch, head)
+    if (g.B == 0) return BRA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
+    if (cudaMemsetAsync(dq, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
+        return BRA_ERR_CUDA;
+    return launch_attend_backward(shape->dtype == BRA_DTYPE_BF16, q, k, v, idx, grad_o, dq, dk, dv, g,
+                                  carve(g, workspace).status, st) == cudaSuccess
                ? BRA_OK
                : BRA_ERR_CUDA;
 }

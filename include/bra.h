@@ -179,6 +179,33 @@ bra_status bra_route_noalloc(const bra_shape* shape, const void* q, const void* 
                              void* stream);
 
 /*
+ * Gradients of bra_attend for a fixed routing (the backward of blog section
+ * 2.2 step 4; top-k has no gradient, so ``idx`` is an input).  With
+ * s_j = <q_t, k_j> / sqrt(d), P = softmax(s) over the union of the routed
+ * regions' tokens (a region listed twice counts once), O = P V and
+ * G = dL/dO:
+ *   dP_j = <G_t, v_j>,  D_t = sum_j P_j dP_j,  dS_j = P_j (dP_j - D_t),
+ *   dQ_t = sum_j dS_j k_j / sqrt(d),  dK_j = sum_t dS_tj q_t / sqrt(d),
+ *   dV_j = sum_t P_tj G_t.
+ * All arithmetic is fp32; dK and dV are accumulated with fp32 atomics, so
+ * their last bits may differ from run to run.
+ *   shape      as for bra_attend; regions of up to about 64 tokens with up
+ *              to 256 routed keys per query fit (staging in shared memory),
+ *              larger ones return BRA_ERR_UNSUPPORTED
+ *   q, k, v    device, [B, H, W, C] of ``shape->dtype``, read only
+ *   idx        device int32 [B, heads, S*S, topk], read only; an entry
+ *              outside [0, S*S) makes the kernel skip that region's
+ *              gradients and record BRA_ERR_BAD_ROUTE in the status block
+ *   grad_o     device, [B, H, W, C] of ``shape->dtype``: dL/dO, read only
+ *   dq, dk, dv device fp32 [B, H, W, C], written (cleared first)
+ *   workspace  as for bra_attend (only its status block is used)
+ * All pointers 16-byte aligned.  Errors: as bra_attend.  Allocates nothing.
+ */
+bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const void* grad_o, float* dq, float* dk, float* dv,
+                               void* workspace, void* stream);
+
+/*
  * Self-test of the failure-detection path (the pages have no counterpart):
  * every kernel that waits on an mbarrier polls it a bounded number of times
  * and, when the limit runs out, records BRA_ERR_TIMEOUT in the workspace

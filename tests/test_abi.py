@@ -77,6 +77,7 @@ def test_bad_shapes_rejected_before_launch(bad, code):
     assert bra._lib.bra_route(ctypes.byref(s), p, p, p, p, None) == code
     assert bra._lib.bra_attend(ctypes.byref(s), p, p, p, p, p, p, None) == code
     assert bra._lib.bra_lce(ctypes.byref(s), p, p, p, p, None) == code
+    assert bra._lib.bra_attend_backward(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
     assert bra.bra_workspace_bytes(s) == 0
 
 
@@ -132,3 +133,20 @@ def test_selftest_rejects_bad_arguments_before_launch():
     assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), ws, (1 << 24) + 1, 0, None) == bra.BRA_ERR_INVALID_ARG
     assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), None, 10, 0, None) == bra.BRA_ERR_INVALID_ARG
     assert bra._lib.bra_selftest_bounded_wait(ctypes.byref(s), ws + 8, 10, 0, None) == bra.BRA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(9))
+def test_backward_null_and_misaligned_pointers(which):
+    s = shp()
+    good = [1 << 20] * 9
+    for bad in (0, (1 << 20) + 8):
+        ptrs = list(good)
+        ptrs[which] = bad
+        assert bra._lib.bra_attend_backward(ctypes.byref(s), *ptrs, None) == bra.BRA_ERR_INVALID_ARG
+
+
+def test_backward_rejects_what_it_cannot_stage():
+    """256-token regions with 1024 routed keys need more shared memory than a CTA has."""
+    s = bra.shape_for(2, 128, 128, 64, 2, 8, 4, "bf16")
+    p = 1 << 20
+    assert bra._lib.bra_attend_backward(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == bra.BRA_ERR_UNSUPPORTED
