@@ -52,6 +52,7 @@ def _bind(path: str):
     lib.oracle_bra_forward.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _dp, _ip, _dp]
     lib.oracle_local_context.argtypes = [_dp, _i, _i, _i, _i, _dp, _dp, _dp]
     lib.oracle_attention_backward.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i, _i, _ip, _dp, _dp, _dp, _dp]
+    lib.oracle_qkv_projection.argtypes = [_dp, _i, _i, _i, _i, _dp, _dp, _dp, _dp, _dp]
     for f in (lib.oracle_region_pool, lib.oracle_region_affinity, lib.oracle_topk_routing,
               lib.oracle_token_attention, lib.oracle_bra_forward):
         f.restype = _i
@@ -177,3 +178,19 @@ def attention_backward(q, k, v, idx, grad_o, heads: int, S: int):
                                              _ptr(dv, _dp)),
            "attention backward")
     return dq, dk, dv
+
+
+def qkv_projection(x, weight, bias=None):
+    """Q, K, V of a feature map X [B, H, W, C]: the three channel chunks of
+    the linear layer ``x @ weight.T + bias`` with ``weight`` [3C, C] and
+    ``bias`` [3C] or None."""
+    x = _f64(x)
+    B, H, W, C = x.shape
+    w = _f64(np.reshape(weight, (3 * C, C)))
+    bb = _f64(np.reshape(bias, (3 * C,))) if bias is not None else None
+    q, k, v = np.zeros_like(x), np.zeros_like(x), np.zeros_like(x)
+    _check(_load().oracle_qkv_projection(_ptr(x, _dp), B, H, W, C, _ptr(w, _dp),
+                                         _ptr(bb, _dp) if bb is not None else None,
+                                         _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp)),
+           "qkv projection")
+    return q, k, v

@@ -13,6 +13,10 @@
  * Routing Attention" (section 3 "Our Approach").  The steps are written out
  * plainly, in the pages' order, with no blocking or fusion:
  *
+ *   0. linear projection: Q, K, V are the three channel chunks of one
+ *      linear layer applied to every token of X (section 2.2 step 2 and
+ *      pseudocode step 2; oracle_qkv_projection, used only by the fused
+ *      projection path);
  *   1. region partition: the H x W map is cut into S x S regions of
  *      n = (H/S)(W/S) tokens (section 2.2 step 1);
  *   2. region-level query/key Q^r, K^r = per-region mean of Q and K
@@ -333,4 +337,29 @@ int oracle_attention_backward(const double* q, const double* k, const double* v,
     free(dp);
     free(key_off);
     return rc;
+}
+
+/* Linear projection (section 2.2 step 2; pseudocode step 2 splits the
+ * output of one linear layer into three equal chunks along the channel axis:
+ * query, key, value).  For every token and output channel o in [0, 3C):
+ *   y[o] = bias[o] + sum_{c < C} w[o][c] * x[c],
+ * and q = y[0, C), k = y[C, 2C), v = y[2C, 3C).  ``w`` is [3C][C] (a linear
+ * layer's [out][in] weight), ``bias`` is [3C] or NULL (no bias: the pages do
+ * not say whether the layer has one).  x, q, k, v are [B, H, W, C] float64;
+ * q, k, v are overwritten. */
+int oracle_qkv_projection(const double* x, int B, int H, int W, int C, const double* w,
+                          const double* bias, double* q, double* k, double* v)
+{
+    if (B < 0 || H <= 0 || W <= 0 || C <= 0) return ORACLE_EINVAL;
+    size_t tokens = (size_t)B * H * W;
+    for (size_t t = 0; t < tokens; ++t) {
+        const double* xt = x + t * C;
+        for (int o = 0; o < 3 * C; ++o) {
+            double acc = bias ? bias[o] : 0.0;
+            for (int c = 0; c < C; ++c) acc += w[(size_t)o * C + c] * xt[c];
+            double* dst = o < C ? q : (o < 2 * C ? k : v);
+            dst[t * C + o % C] = acc;
+        }
+    }
+    return 0;
 }

@@ -120,3 +120,33 @@ def test_backward_pins_catch_mutation(tmp_path, name, old, new):
             except AssertionError:
                 failures += 1
     assert failures > 0, f"no pin caught mutation {name}"
+
+
+# The projection's pins catch slips in its own function.
+QKV_MUTATIONS = [
+    ("qkv_weight_transposed", "acc += w[(size_t)o * C + c] * xt[c];", "acc += w[(size_t)c * 3 * C + o] * xt[c];"),
+    ("qkv_bias_dropped", "double acc = bias ? bias[o] : 0.0;", "double acc = 0.0;"),
+    ("qkv_chunks_swapped", "double* dst = o < C ? q : (o < 2 * C ? k : v);",
+     "double* dst = o < C ? k : (o < 2 * C ? q : v);"),
+    ("qkv_channels_reversed", "dst[t * C + o % C] = acc;", "dst[t * C + (C - 1 - o % C)] = acc;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", QKV_MUTATIONS, ids=[m[0] for m in QKV_MUTATIONS])
+def test_projection_pins_catch_mutation(tmp_path, name, old, new):
+    import test_oracle_qkv as pins
+    lib = build_variant(tmp_path, name, old, new)
+    checks = [
+        pins.test_block_identity_weights_give_scaled_copies,
+        pins.test_bias_only_fills_each_chunk_with_its_bias,
+        pins.test_permutation_rows_select_input_channels,
+        lambda: pins.test_matches_numpy_matmul(True),
+    ]
+    failures = 0
+    with oracle.swapped_library(lib):
+        for check in checks:
+            try:
+                check()
+            except AssertionError:
+                failures += 1
+    assert failures > 0, f"no pin caught mutation {name}"
