@@ -6,6 +6,12 @@ C=64, 2 heads of 32, S=7 (49 regions of 8x8 tokens), topk=1, bf16, seeded
 synthetic inputs.  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--lce] [--qkv]
+
+``--qkv`` starts every step from the feature map X instead of Q, K, V: the
+fused projection (Q, K, V and their region means in one kernel), routing on
+those means and attention (bra_forward_qkv), with seeded linear-layer
+weights; the roofline then also reports the projection kernel.
 
 N > 1 runs under torch.distributed.run, one process per GPU, each rank an
 independent replica on its own batch (the path has no exchange step), and
@@ -48,6 +54,16 @@ TRAFFIC_RECORDS: dict[str, float] = {
 }
 
 
+# DRAM bytes per launch of the fused projection kernel on the stage-1 workload
+# (same rule as above, keyed by kernel_sources_hash("qkv")).  Most of the
+# 77 MB of Q, K, V it writes is still dirty in L2 when the launch ends, so the
+# figure is below the algorithmic bytes.
+QKV_TRAFFIC_RECORDS: dict[str, float] = {
+    # ncu --set full capture of bra_qkv_kernel<1>: dram read 25.77 MB + write 19.86 MB
+    "b2ea237c13991f40d6976715f56941fb6f38a5fff2805933a79d9a090ff350f5": 45.62944e6,
+}
+
+
 def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -59,6 +75,8 @@ def parse(argv=None):
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--lce", action="store_true",
                    help="add the local context enhancement (bra_lce, seeded 5x5 depthwise weights) to every step")
+    p.add_argument("--qkv", action="store_true",
+                   help="start every step from the feature map: fused Q/K/V projection + routing + attention")
     return p.parse_args(argv)
 
 
@@ -83,6 +101,10 @@ def byte_counts(shape: bi.BraShape) -> dict:
         "attend": 4 * m + idx,
         # pooling kernel: Q, K read, means written
         "pool": 2 * m + 2 * means,
+        # fused projection: X and the layer read, Q, K, V and the means written
+        "qkv": 4 * m + 2 * means + 3 * shape.C * shape.C * es + 3 * shape.C * 4,
+        # the path from X: X read, O and I^r written
+        "path_min_qkv": 2 * m + idx,
     }
 
 
@@ -100,11 +122,13 @@ def measured_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_hash() -> str:
+def kernel_sources_hash(prefix: str = "attend") -> str:
+    """sha256 of the sources of the kernel named by ``prefix`` (its own files,
+    the TMA host code and the shared device headers)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dynamic_sparse_attention_bra_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith(("attend", "tma_host")) or name in ("common.cuh", "kernels.h", "tc_ptx.cuh"):
+        if name.startswith((prefix, "tma_host")) or name in ("common.cuh", "kernels.h", "tc_ptx.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()
@@ -163,10 +187,11 @@ class ClockSampler:
 
 
 def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
-                          batches_per_call: int | None = None) -> dict:
+                          batches_per_call: int | None = None, from_feature_map: bool = False) -> dict:
     """The float64 oracle (single thread) on bounded samples of the workload."""
     import oracle
     inp = bi.make_inputs(shape, seed)
+    proj = bi.make_projection_inputs(shape, seed) if from_feature_map else None
     bpc = batches_per_call or shape.B
     tokens = 0
     t0 = time.perf_counter()
@@ -174,7 +199,11 @@ def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
     while True:
         b0 = (calls * bpc) % shape.B
         sl = slice(b0, b0 + bpc)
-        oracle.bra_forward(inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl], shape.heads, shape.S, shape.topk)
+        if proj is not None:
+            q, k, v = oracle.qkv_projection(proj.x_f64[sl], proj.w_f64, proj.b_f64)
+        else:
+            q, k, v = inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl]
+        oracle.bra_forward(q, k, v, shape.heads, shape.S, shape.topk)
         tokens += bpc * shape.H * shape.W
         calls += 1
         el = time.perf_counter() - t0
@@ -220,6 +249,7 @@ def run_reference(args):
     shape, seed = bi.WORKLOADS[args.workload]
     import oracle
     inp = bi.make_inputs(shape, seed)
+    proj = bi.make_projection_inputs(shape, seed) if args.qkv else None
     bpc = 1  # one image per step: a bounded sample of the batch
     lce_w = lce_b = None
     if args.lce:
@@ -229,9 +259,13 @@ def run_reference(args):
 
     def step(i):
         sl = slice(i % shape.B, i % shape.B + bpc)
-        o, _ = oracle.bra_forward(inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl], shape.heads, shape.S, shape.topk)
+        if args.qkv:
+            q, k, v = oracle.qkv_projection(proj.x_f64[sl], proj.w_f64, proj.b_f64)
+        else:
+            q, k, v = inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl]
+        o, _ = oracle.bra_forward(q, k, v, shape.heads, shape.S, shape.topk)
         if args.lce:
-            o = o + oracle.local_context(inp.v_f64[sl], lce_w, lce_b)
+            o = o + oracle.local_context(v, lce_w, lce_b)
         return o
     for i in range(args.warmup):
         step(i)
@@ -247,7 +281,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {**workload_config(shape, args.workload), "sample_images_per_step": bpc,
-                   "local_context": bool(args.lce)},
+                   "local_context": bool(args.lce), "from_feature_map": bool(args.qkv)},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"{bpc} of {shape.B} images per step, float64 oracle, one thread"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -279,7 +313,13 @@ def run_ours(args):
 
     host_qkv = [host(a).pin_memory() for a in (inp.q_store, inp.k_store, inp.v_store)]
     cnt = byte_counts(shape)
-    set_bytes = 4 * cnt["map"] + cnt["idx"]
+    set_bytes = (5 if args.qkv else 4) * cnt["map"] + cnt["idx"]
+    proj = host_x = w_qkv = b_qkv = None
+    if args.qkv:
+        proj = bi.make_projection_inputs(shape, rank_seed(seed, rank))
+        host_x = host(proj.x_store).pin_memory()
+        w_qkv = host(proj.w_store).to(dev)
+        b_qkv = torch.from_numpy(proj.b_store).to(dev)
     nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
     s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
     sets = []
@@ -289,6 +329,10 @@ def run_ours(args):
             q=q, k=k, v=v, o=torch.empty_like(q),
             idx=torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device=dev),
             ws=torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device=dev)))
+        if args.qkv:
+            sets[-1]["x"] = host_x.to(dev)
+            sets[-1]["qr"] = torch.empty((shape.B, shape.heads, shape.R, shape.d), device=dev)
+            sets[-1]["kr"] = torch.empty_like(sets[-1]["qr"])
     stream = torch.cuda.Stream(device=dev)
     sp = stream.cuda_stream
 
@@ -299,11 +343,16 @@ def run_ours(args):
         lce_w = (torch.randn(shape.C * 25, generator=g) / 5.0).to(dev)
         lce_b = torch.randn(shape.C, generator=g).to(dev)
 
-    def step(i):
-        b = sets[i % nsets]
-        bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+    def forward(b):
+        if args.qkv:
+            bra.bra_forward_qkv(s, b["x"], w_qkv, b_qkv, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+        else:
+            bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
         if args.lce:
             bra.bra_lce(s, b["v"], lce_w, lce_b, b["o"], sp)
+
+    def step(i):
+        forward(sets[i % nsets])
 
     for i in range(args.warmup):
         step(i)
@@ -317,6 +366,8 @@ def run_ours(args):
     # launches ends their overlap, so this pass is not the step time).
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    ev_qkv = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] if args.qkv else []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         if world > 1:
@@ -333,6 +384,11 @@ def run_ours(args):
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 b = sets[i % nsets]
+                if args.qkv:
+                    ev_qkv[i][0].record(stream)
+                    bra.bra_qkv_project(s, b["x"], w_qkv, b_qkv, b["q"], b["k"], b["v"], b["qr"], b["kr"],
+                                        b["ws"], sp)
+                    ev_qkv[i][1].record(stream)
                 bra.bra_route(s, b["q"], b["k"], b["idx"], b["ws"], sp)
                 ev[i][0].record(stream)
                 bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
@@ -342,6 +398,7 @@ def run_ours(args):
         torch.distributed.barrier()
     total_ms = start.elapsed_time(end)
     attend_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    qkv_ms = sum(a.elapsed_time(b) for a, b in ev_qkv) / args.steps if args.qkv else 0.0
     for b in sets:
         st = bra.bra_device_status(s, b["ws"], sp)
         if st != bra.BRA_OK:
@@ -352,16 +409,17 @@ def run_ours(args):
     o_host = torch.empty(host_qkv[0].shape, dtype=tdt).pin_memory()
     idx_host = torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32).pin_memory()
     b0 = sets[0]
-    h2d = 3 * cnt["map"]
+    h2d = (1 if args.qkv else 3) * cnt["map"]
     d2h = cnt["map"] + cnt["idx"]
 
     def e2e_step():
         with torch.cuda.stream(stream):
-            for dst, src in zip((b0["q"], b0["k"], b0["v"]), host_qkv):
-                dst.copy_(src, non_blocking=True)
-            bra.bra_forward(s, b0["q"], b0["k"], b0["v"], b0["o"], b0["idx"], b0["ws"], sp)
-            if args.lce:
-                bra.bra_lce(s, b0["v"], lce_w, lce_b, b0["o"], sp)
+            if args.qkv:
+                b0["x"].copy_(host_x, non_blocking=True)
+            else:
+                for dst, src in zip((b0["q"], b0["k"], b0["v"]), host_qkv):
+                    dst.copy_(src, non_blocking=True)
+            forward(b0)
             o_host.copy_(b0["o"], non_blocking=True)
             idx_host.copy_(b0["idx"], non_blocking=True)
 
@@ -378,7 +436,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
 
-    total_ms, attend_ms, e2e_ms = max_over_ranks([total_ms, attend_ms, e2e_ms], world, dev)
+    total_ms, attend_ms, e2e_ms, qkv_ms = max_over_ranks([total_ms, attend_ms, e2e_ms, qkv_ms], world, dev)
     ms_per_step = total_ms / args.steps
     tokens = shape.tokens * world
     value = whole_job_tokens_per_s(shape.tokens, world, ms_per_step)
@@ -386,6 +444,7 @@ def run_ours(args):
     if rank == 0:
         peak, peak_kind = measured_peaks()
         achieved = cnt["attend"] / (attend_ms * 1e-3) / 1e9
+        path_key = "path_min_qkv" if args.qkv else "path_min"
         digest = kernel_sources_hash()
         traffic = TRAFFIC_RECORDS.get(digest)
         line = {
@@ -394,7 +453,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": shape.dtype, "data": "synthetic",
             "config": {**workload_config(shape, args.workload), "parallelism": f"replicas{world}",
-                       "local_context": bool(args.lce),
+                       "local_context": bool(args.lce), "from_feature_map": bool(args.qkv),
                        "l2": f"rotating {nsets} input sets ({nsets * set_bytes / 2**20:.0f} MiB) > 126 MiB L2"},
             "roofline": {
                 "kernel": "bra_attend", "bound": "hbm", "achieved": achieved, "peak": peak,
@@ -402,17 +461,25 @@ def run_ours(args):
                 "algorithmic_bytes": cnt["attend"], "launch_ms": attend_ms,
             },
             "path_roofline": {
-                "min_bytes": cnt["path_min"], "flops": attention_flops(shape),
+                "min_bytes": cnt[path_key], "flops": attention_flops(shape),
                 "time_us": ms_per_step * 1e3,
-                "frac": cnt["path_min"] / peak / 1e9 / (ms_per_step * 1e-3),
+                "frac": cnt[path_key] / peak / 1e9 / (ms_per_step * 1e-3),
             },
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": (4 if args.lce else 3) * args.steps,
             "clocks": clocks.report(),
         }
+        if args.qkv:
+            qkv_gbs = cnt["qkv"] / (qkv_ms * 1e-3) / 1e9
+            line["qkv_roofline"] = {
+                "kernel": "bra_qkv_project", "bound": "hbm", "achieved": qkv_gbs, "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": qkv_gbs / peak,
+                "traffic": QKV_TRAFFIC_RECORDS.get(kernel_sources_hash("qkv")),
+                "algorithmic_bytes": cnt["qkv"], "launch_ms": qkv_ms,
+            }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_throughput(shape, seed)
+            line["cpu_baseline"] = cpu_oracle_throughput(shape, seed, from_feature_map=args.qkv)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

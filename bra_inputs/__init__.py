@@ -21,6 +21,12 @@ applied to ``key(seed, stream) + (i + 1) * 0x9E3779B97F4A7C15`` for element
 counter ``i``, turned into doubles in (0, 1) with 53 random bits and into
 normals with the Box-Muller transform (pairs (2j, 2j+1) give cos/sin).
 Streams: Q = 0, K = 1, V = 2; means and noise use sub-streams 0 and 1.
+
+Projection workloads (the Q, K, V linear layer in front of the path) draw
+the feature map X with the same recipe on stream 3, and the layer's
+parameters the way a freshly initialised linear layer holds them:
+W [3C, C] and b [3C] uniform in (-1/sqrt(C), 1/sqrt(C)), from the uniform
+streams 8 (W) and 9 (b).
 """
 from __future__ import annotations
 
@@ -214,3 +220,27 @@ def make_inputs(shape: BraShape, seed: int) -> BraInputs:
     (bf16 workloads) rounded to bfloat16."""
     stores = [_store(feature_map(shape, seed, stream), shape.dtype) for stream in (0, 1, 2)]
     return BraInputs(shape, *stores)
+
+
+class ProjectionInputs:
+    """X [B, H, W, C] and W [3C, C] as bfloat16 bit patterns (int16), b [3C]
+    as float32, plus their exact float64 widenings for the oracle."""
+
+    def __init__(self, shape: BraShape, x_store, w_store, b_store):
+        self.shape = shape
+        self.x_store, self.w_store, self.b_store = x_store, w_store, b_store
+        self.x_f64 = bf16_bits_to_f64(x_store)
+        self.w_f64 = bf16_bits_to_f64(w_store)
+        self.b_f64 = b_store.astype(np.float64)
+
+
+def make_projection_inputs(shape: BraShape, seed: int) -> ProjectionInputs:
+    """Feature map and linear-layer parameters for the fused projection."""
+    if shape.dtype != "bf16":
+        raise ValueError("the projection workloads are bf16")
+    C = shape.C
+    bound = 1.0 / np.sqrt(C)
+    x = _store(feature_map(shape, seed, 3), "bf16")
+    w = _store(((2.0 * uniform01(seed, 8, 3 * C * C) - 1.0) * bound).reshape(3 * C, C), "bf16")
+    b = ((2.0 * uniform01(seed, 9, 3 * C) - 1.0) * bound).astype(np.float32)
+    return ProjectionInputs(shape, x, w, b)

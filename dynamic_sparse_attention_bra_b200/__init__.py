@@ -26,7 +26,7 @@ __all__ = [
     "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
     "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
     "bra_route_noalloc", "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward",
-    "EXPORTED_SYMBOLS",
+    "bra_qkv_project", "bra_forward_qkv", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +37,8 @@ BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
                     "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc",
-                    "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward")
+                    "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward", "bra_qkv_project",
+                    "bra_forward_qkv")
 NOALLOC_MAX_MEANS = 1 << 20  # BRA_NOALLOC_MAX_MEANS
 
 
@@ -68,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.bra_lce.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.bra_selftest_bounded_wait.argtypes = [sp, vp, ctypes.c_uint, ctypes.c_int, vp]
     lib.bra_attend_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.bra_qkv_project.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.bra_forward_qkv.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_device_status.argtypes = [sp, vp, vp]
     lib.bra_route_noalloc.argtypes = [sp, vp, vp, vp, vp]
     lib.bra_route_noalloc.restype = ctypes.c_int
@@ -134,6 +137,20 @@ def bra_attend_backward(shape: BraShape, q, k, v, idx, grad_o, dq, dk, dv, works
     _check(_lib.bra_attend_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(grad_o),
                                     _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream)),
            "bra_attend_backward")
+
+
+def bra_qkv_project(shape: BraShape, x, w_qkv, b_qkv, q, k, v, q_r, k_r, workspace, stream=None) -> None:
+    """[q | k | v] = x w_qkv^T (+ b_qkv) in bf16 and the fp32 region means q_r, k_r of q and k."""
+    _check(_lib.bra_qkv_project(ctypes.byref(shape), _ptr(x), _ptr(w_qkv), _ptr(b_qkv) if b_qkv is not None else None,
+                                _ptr(q), _ptr(k), _ptr(v), _ptr(q_r), _ptr(k_r), _ptr(workspace), _stream(stream)),
+           "bra_qkv_project")
+
+
+def bra_forward_qkv(shape: BraShape, x, w_qkv, b_qkv, q, k, v, o, idx, workspace, stream=None) -> None:
+    """The path from the feature map x: projection with region means, routing, attention."""
+    _check(_lib.bra_forward_qkv(ctypes.byref(shape), _ptr(x), _ptr(w_qkv), _ptr(b_qkv) if b_qkv is not None else None,
+                                _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(idx), _ptr(workspace), _stream(stream)),
+           "bra_forward_qkv")
 
 
 def bra_selftest_bounded_wait(shape: BraShape, workspace, tries: int, arrive: bool, stream=None) -> None:

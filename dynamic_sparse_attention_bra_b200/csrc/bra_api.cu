@@ -11,6 +11,7 @@
 #include "backward.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "qkv.h"
 
 namespace bra {
 namespace {
@@ -204,6 +205,40 @@ bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void
                                   carve(g, workspace).status, st) == cudaSuccess
                ? BRA_OK
                : BRA_ERR_CUDA;
+}
+
+bra_status bra_qkv_project(const bra_shape* shape, const void* x, const void* w_qkv, const float* b_qkv, void* q,
+                           void* k, void* v, float* q_r, float* k_r, void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!x || !w_qkv || !q || !k || !v || !q_r || !k_r || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_qkv) || (b_qkv && !aligned16(b_qkv)) || !aligned16(q) || !aligned16(k) ||
+        !aligned16(v) || !aligned16(q_r) || !aligned16(k_r) || !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    if (shape->dtype != BRA_DTYPE_BF16 || qkv_check(g) != BRA_OK) return BRA_ERR_UNSUPPORTED;
+    if (g.B == 0) return BRA_OK;
+    return qkv_launch(g, x, w_qkv, b_qkv, q, k, v, q_r, k_r, carve(g, workspace).status,
+                      static_cast<cudaStream_t>(stream));
+}
+
+bra_status bra_forward_qkv(const bra_shape* shape, const void* x, const void* w_qkv, const float* b_qkv, void* q,
+                           void* k, void* v, void* o, int32_t* idx, void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!x || !w_qkv || !q || !k || !v || !o || !idx || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_qkv) || (b_qkv && !aligned16(b_qkv)) || !aligned16(q) || !aligned16(k) ||
+        !aligned16(v) || !aligned16(o) || !aligned16(idx) || !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    if (shape->dtype != BRA_DTYPE_BF16 || qkv_check(g) != BRA_OK) return BRA_ERR_UNSUPPORTED;
+    if (g.B == 0) return BRA_OK;
+    const Workspace w = carve(g, workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = qkv_launch(g, x, w_qkv, b_qkv, q, k, v, w.qr, w.kr, w.status, st);
+    if (rc != BRA_OK) return rc;
+    if (launch_route(w.qr, w.kr, idx, g, st) != cudaSuccess) return BRA_ERR_CUDA;
+    return attend_impl(shape, g, q, k, v, idx, o, w, st);
 }
 
 bra_status bra_selftest_bounded_wait(const bra_shape* shape, void* workspace, unsigned int tries, int arrive,

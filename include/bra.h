@@ -206,6 +206,41 @@ bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void
                                void* workspace, void* stream);
 
 /*
+ * Linear projection fused with the region means (blog "BiFormer Reshapes
+ * Visual Attention with Bi-Level Routing", Part 2 section 2.2 step 2 and
+ * pseudocode step 2, where query, key and value are the three channel chunks
+ * of one linear layer; step 3's Q^r, K^r follow in the same pass).  For every
+ * token x (C channels) and output channel o in [0, 3C):
+ *   y[o] = bias[o] + sum_c w_qkv[o][c] * x[c],
+ * q = y[0, C), k = y[C, 2C), v = y[2C, 3C), each rounded to bf16 from the
+ * fp32 accumulator; q_r and k_r are the fp32 means of the stored (bf16) q
+ * and k over every region, exactly what bra_route pools from them.
+ *   shape      dtype BRA_DTYPE_BF16, C = 64 or 128, regions of at most 128
+ *              tokens; other valid shapes return BRA_ERR_UNSUPPORTED (topk
+ *              is only checked)
+ *   x          device bf16 [B, H, W, C], read only
+ *   w_qkv      device bf16 [3C][C] (a linear layer's [out][in] weight), read only
+ *   b_qkv      device fp32 [3C], or NULL for no bias
+ *   q, k, v    device bf16 [B, H, W, C], written; they must not overlap x
+ *   q_r, k_r   device fp32 [B, heads, S*S, d], written
+ *   workspace  as for bra_route (only its status block is used: a device
+ *              wait that gives up records BRA_ERR_TIMEOUT there)
+ * All pointers 16-byte aligned.  Errors: BRA_ERR_INVALID_ARG (bad shape,
+ * NULL or misaligned pointer), BRA_ERR_UNSUPPORTED, BRA_ERR_CUDA.
+ */
+bra_status bra_qkv_project(const bra_shape* shape, const void* x, const void* w_qkv, const float* b_qkv, void* q,
+                           void* k, void* v, float* q_r, float* k_r, void* workspace, void* stream);
+
+/*
+ * The whole path from the feature map: bra_qkv_project (its region means go
+ * to the workspace), the top-k routing of bra_route on those means, then
+ * bra_attend.  Writes q, k, v (kept for a backward pass), ``idx`` and ``o``.
+ * Arguments and limits as for bra_qkv_project and bra_forward.
+ */
+bra_status bra_forward_qkv(const bra_shape* shape, const void* x, const void* w_qkv, const float* b_qkv, void* q,
+                           void* k, void* v, void* o, int32_t* idx, void* workspace, void* stream);
+
+/*
  * Self-test of the failure-detection path (the pages have no counterpart):
  * every kernel that waits on an mbarrier polls it a bounded number of times
  * and, when the limit runs out, records BRA_ERR_TIMEOUT in the workspace

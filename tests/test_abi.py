@@ -78,6 +78,8 @@ def test_bad_shapes_rejected_before_launch(bad, code):
     assert bra._lib.bra_attend(ctypes.byref(s), p, p, p, p, p, p, None) == code
     assert bra._lib.bra_lce(ctypes.byref(s), p, p, p, p, None) == code
     assert bra._lib.bra_attend_backward(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
+    assert bra._lib.bra_qkv_project(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
+    assert bra._lib.bra_forward_qkv(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
     assert bra.bra_workspace_bytes(s) == 0
 
 
@@ -150,3 +152,32 @@ def test_backward_rejects_what_it_cannot_stage():
     s = bra.shape_for(2, 128, 128, 64, 2, 8, 4, "bf16")
     p = 1 << 20
     assert bra._lib.bra_attend_backward(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == bra.BRA_ERR_UNSUPPORTED
+
+
+# Pointer order of bra_qkv_project after the shape: x, w_qkv, b_qkv, q, k, v,
+# q_r, k_r, workspace; b_qkv may be NULL (no bias) but not misaligned.
+@pytest.mark.parametrize("which", range(9))
+def test_projection_null_and_misaligned_pointers(which):
+    s = bra.shape_for(2, 56, 56, 64, 2, 7, 1, "bf16")
+    good = [1 << 20] * 9
+    for bad in (0, (1 << 20) + 8):
+        if which == 2 and bad == 0:
+            continue
+        ptrs = list(good)
+        ptrs[which] = bad
+        assert bra._lib.bra_qkv_project(ctypes.byref(s), *ptrs, None) == bra.BRA_ERR_INVALID_ARG
+        # bra_forward_qkv: x, w, b, q, k, v, o, idx, workspace
+        assert bra._lib.bra_forward_qkv(ctypes.byref(s), *ptrs, None) == bra.BRA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args", [
+    (64, 14, 14, 256, 8, 7, 16, "bf16"),   # C = 256: weights do not stay resident in shared memory
+    (2, 128, 128, 64, 2, 8, 4, "bf16"),    # 256-token regions exceed one 128-row tile
+    (2, 56, 56, 64, 2, 7, 1, "f32"),       # the projection runs on bf16 tensor cores only
+    (2, 56, 56, 96, 3, 7, 1, "bf16"),      # C not a multiple of 64
+])
+def test_projection_rejects_what_it_does_not_cover(args):
+    s = bra.shape_for(*args)
+    p = 1 << 20
+    assert bra._lib.bra_qkv_project(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == bra.BRA_ERR_UNSUPPORTED
+    assert bra._lib.bra_forward_qkv(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == bra.BRA_ERR_UNSUPPORTED
