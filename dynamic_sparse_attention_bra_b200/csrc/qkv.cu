@@ -38,7 +38,7 @@
 namespace bra {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;    // two warpgroups over the 128 TMEM lanes
 constexpr int kRows = 128;          // MMA M: tokens per tile
 constexpr int kNChunk = 192;        // MMA N per instruction
 constexpr int kBlockBytes = kRows * 128;  // one 64-channel block of 128 token rows
@@ -78,7 +78,7 @@ bool make_qkv_plan(const Geometry& g, QkvPlan* p) {
     // Pooling items: 8 chunks x parts x (Q and K blocks) x regions per tile.
     const int base = 8 * 2 * (g.C / 64) * p->nrx * p->nry;
     p->parts = 1;
-    while (p->parts < 4 && base * p->parts * 2 <= kThreads && p->parts * 2 <= g.n) p->parts *= 2;
+    while (p->parts < 4 && base * p->parts * 2 <= kRows && p->parts * 2 <= g.n) p->parts *= 2;
     return true;
 }
 
@@ -91,7 +91,8 @@ struct Layout {
     static constexpr int kOffA = kOffW + kWBytes;      // [stages][KB][128 rows][128 B]
     static constexpr int kOffOut = kOffA + kAStages * KB * kBlockBytes;  // [3][KB][128 rows][128 B]
     static constexpr int kOffBias = kOffOut + 3 * KB * kBlockBytes;
-    static constexpr int kOffMisc = kOffBias + 3 * C * 4;
+    static constexpr int kOffScratch = kOffBias + 3 * C * 4;  // [128][8] fp32 partial sums (C = 64 only)
+    static constexpr int kOffMisc = kOffScratch + (KB == 1 ? kRows * 8 * 4 : 0);
     static constexpr int kBytes = kOffMisc + 48;  // afull[2], wfull, mma_done, TMEM slot
     static constexpr int kAlloc = kBytes + 1024;       // room to align the base to 1 KB
     static constexpr uint32_t kTmemCols = KB == 1 ? 256 : 512;
@@ -121,6 +122,28 @@ __device__ __forceinline__ TileCoord tile_coord(long long t, const QkvPlan& p) {
     return {b, tx * p.bw, ty * p.bh};
 }
 
+// Two fp32 lanes in one 64-bit register (x in the low half), added with one
+// add.rn.f32x2 (sm_100a), each lane rounded as a scalar fp32 add would be.
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+    return f;
+}
+// bf16 pair -> packed fp32 pair (a bf16 is the high half of its float)
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t r) {
+    return f2_pack(__uint_as_float(r << 16), __uint_as_float(r & 0xffff0000u));
+}
+
 template <int KB>
 __global__ void __launch_bounds__(kThreads, Layout<KB>::kCtasPerSm)
 bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
@@ -135,12 +158,14 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
     const uint32_t sbase = ptx::smem_addr(smem);
     const uint32_t sW = sbase + L::kOffW, sA = sbase + L::kOffA, sOut = sbase + L::kOffOut;
     float* bias_s = reinterpret_cast<float*>(smem + L::kOffBias);
+    float* scratch = reinterpret_cast<float*>(smem + L::kOffScratch);  // [128 items][8]
     uint64_t* afull = reinterpret_cast<uint64_t*>(smem + L::kOffMisc);  // [kStages]
     uint64_t* wfull = afull + 2;
     uint64_t* mma_done = afull + 3;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc + 32);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, wg = warp >> 2;  // TMEM lane quadrant, warpgroup
     const uint32_t a_bytes = (uint32_t)KB * 64 * p.rows * 2;
 
     // ---- set-up ------------------------------------------------------------------
@@ -194,13 +219,9 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
         for (int j = 0; j < kStages; ++j) issue_x(j);
     }
 
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int row = tid;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const int row = tid & (kRows - 1);
     const float inv_n = 1.f / (float)g.n;
-    // Pooling item of this thread: 16-byte chunk ``pc`` (8 channels) of one
-    // 64-channel block, token part ``pp`` (tokens pp, pp + parts, ...), block
-    // and region from the higher bits.  Eight consecutive lanes read the
-    // eight chunks of one token row: conflict-free 16-byte loads.
     const int parts = p.parts;
     const int pc = lane & 7;
     const int items = 8 * parts * 2 * KB * p.nrx * p.nry;
@@ -262,20 +283,28 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
         __syncthreads();
 
         // ---- epilogue: row -> +bias -> bf16 -> swizzled staging ---------------
+        // Warpgroup wg takes output columns [wg * 3C/2, (wg + 1) * 3C/2) of its
+        // rows, 32 columns (four 16-byte chunks of one staging row) at a time.
 #pragma unroll
-        for (int c0 = 0; c0 < 3 * C; c0 += 64) {
-            uint32_t r[64];
-            ptx::tmem_ld64(tmem + lane_base + c0, r);
-            const int o = c0 / C, cin = c0 - o * C, kb = cin >> 6;
+        for (int k32 = 0; k32 < 3 * C / 64; ++k32) {
+            const int c0 = wg * (3 * C / 2) + k32 * 32;
+            uint32_t r[32];
+            ptx::tmem_ld32(tmem + lane_base + c0, r);
+            ptx::tmem_ld_wait();
+            const int o = c0 / C, cin = c0 - o * C, kb = cin >> 6, ch0 = (cin & 63) >> 3;
             const uint32_t dst = sOut + (o * KB + kb) * kBlockBytes + row * 128;
             const float4* b4 = reinterpret_cast<const float4*>(bias_s + c0);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const float4 ba = b4[2 * ch], bb = b4[2 * ch + 1];
-                const float* f = reinterpret_cast<const float*>(&r[ch * 8]);
-                ptx::st_shared_v4(dst + ((ch ^ (row & 7)) << 4), ptx::pack_bf16x2(f[0] + ba.x, f[1] + ba.y),
-                                  ptx::pack_bf16x2(f[2] + ba.z, f[3] + ba.w), ptx::pack_bf16x2(f[4] + bb.x, f[5] + bb.y),
-                                  ptx::pack_bf16x2(f[6] + bb.z, f[7] + bb.w));
+            for (int cc = 0; cc < 4; ++cc) {
+                const float4 ba = b4[2 * cc], bb = b4[2 * cc + 1];
+                const uint32_t* q = r + cc * 8;
+                const float2 s0 = f2_unpack(f2_add(f2_pack(__uint_as_float(q[0]), __uint_as_float(q[1])), f2_pack(ba.x, ba.y)));
+                const float2 s1 = f2_unpack(f2_add(f2_pack(__uint_as_float(q[2]), __uint_as_float(q[3])), f2_pack(ba.z, ba.w)));
+                const float2 s2 = f2_unpack(f2_add(f2_pack(__uint_as_float(q[4]), __uint_as_float(q[5])), f2_pack(bb.x, bb.y)));
+                const float2 s3 = f2_unpack(f2_add(f2_pack(__uint_as_float(q[6]), __uint_as_float(q[7])), f2_pack(bb.z, bb.w)));
+                ptx::st_shared_v4(dst + (((ch0 + cc) ^ (row & 7)) << 4), ptx::pack_bf16x2(s0.x, s0.y),
+                                  ptx::pack_bf16x2(s1.x, s1.y), ptx::pack_bf16x2(s2.x, s2.y),
+                                  ptx::pack_bf16x2(s3.x, s3.y));
             }
         }
         ptx::fence_proxy_async_smem();
@@ -292,49 +321,81 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
         }
 
         // ---- region means of the staged Q and K ---------------------------------
-        // Item e: chunk pc = e % 8, part pp = (e / 8) % parts, block
-        // (Q or K, 64-channel block) and region above.  Every lane of a warp
-        // takes part in the shuffles (items past the end add zeros).
+        // Item e: chunk pc = e % 8 (8 channels), part pp = (e / 8) % parts,
+        // block (Q or K, 64-channel block) and region above.  A thread sums its
+        // chunk over tokens first, first + stride, ... of the region; parts are
+        // lanes 8 apart and are folded with shuffles (every lane of the warp
+        // takes part; items past the end add zeros).  Eight consecutive lanes
+        // read the eight chunks of one token row: conflict-free 16-byte loads.
         const int rx0 = tc.x0 / g.ws, ry0 = tc.y0 / g.hs;
-        for (int e0 = warp * 32; e0 < items; e0 += kThreads) {
-            const int e = e0 + lane;
+        auto region_sum = [&](int e, int first, int stride, float (&out)[8], float*& dst) -> bool {
             const int pp = (e >> 3) % parts;
             const int rest = (e >> 3) / parts;
             const int blk = rest % (2 * KB), reg = rest / (2 * KB);
             const int j = reg / p.nrx, i = reg - j * p.nrx;
             const int rx = rx0 + i, ry = ry0 + j;
             const bool live = e < items && rx < g.S && ry < g.S;
-            float acc[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-            if (live) {
-                const uint8_t* buf = smem + L::kOffOut + blk * kBlockBytes;  // blocks 0..KB-1: Q, KB..2KB-1: K
-                const int tbase = j * g.hs * p.bw + i * g.ws;
-#pragma unroll 4
-                for (int ti = pp; ti < g.n; ti += parts) {
-                    const int yi = ti / g.ws, xi = ti - yi * g.ws;
-                    const int t = tbase + yi * p.bw + xi;
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+            int ti = pp + first;
+            if (live && ti < g.n) {
+                const uint8_t* buf = smem + L::kOffOut + blk * kBlockBytes;  // blocks 0..KB-1: Q, then K
+                int yi = ti / g.ws, xi = ti - yi * g.ws;
+                int t = (j * g.hs + yi) * p.bw + i * g.ws + xi;
+                for (; ti < g.n; ti += stride) {
                     const uint4 v = *reinterpret_cast<const uint4*>(buf + t * 128 + ((pc ^ (t & 7)) << 4));
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        acc[2 * c] += __uint_as_float(w[c] << 16);
-                        acc[2 * c + 1] += __uint_as_float(w[c] & 0xffff0000u);
+                    acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
+                    acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
+                    acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
+                    acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
+                    t += stride;
+                    xi += stride;
+                    while (xi >= g.ws) {
+                        xi -= g.ws;
+                        t += p.bw - g.ws;
                     }
                 }
             }
-            // Parts are lanes 8 apart: fold them onto part 0.
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float2 f = f2_unpack(acc[c]);
+                out[2 * c] = f.x;
+                out[2 * c + 1] = f.y;
+            }
             for (int off = 8; off < 8 * parts; off <<= 1)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], off);
-            if (live && pp == 0) {
-                const int o = blk / KB, cin = (blk - o * KB) * 64 + pc * 8;
-                float* dst = (o == 0 ? qr : kr) +
-                             (((size_t)tc.b * g.heads + (cin >> 5)) * g.R + ry * g.S + rx) * 32 + (cin & 31);
-                reinterpret_cast<float4*>(dst)[0] =
-                    make_float4(acc[0] * inv_n, acc[1] * inv_n, acc[2] * inv_n, acc[3] * inv_n);
-                reinterpret_cast<float4*>(dst)[1] =
-                    make_float4(acc[4] * inv_n, acc[5] * inv_n, acc[6] * inv_n, acc[7] * inv_n);
+                for (int c = 0; c < 8; ++c) out[c] += __shfl_xor_sync(0xffffffffu, out[c], off);
+            const int o = blk / KB, cin = (blk - o * KB) * 64 + pc * 8;
+            dst = (o == 0 ? qr : kr) + (((size_t)tc.b * g.heads + (cin >> 5)) * g.R + ry * g.S + rx) * 32 + (cin & 31);
+            return live && pp == 0;
+        };
+        auto store_mean = [&](float* dst, const float (&s)[8]) {
+            reinterpret_cast<float4*>(dst)[0] = make_float4(s[0] * inv_n, s[1] * inv_n, s[2] * inv_n, s[3] * inv_n);
+            reinterpret_cast<float4*>(dst)[1] = make_float4(s[4] * inv_n, s[5] * inv_n, s[6] * inv_n, s[7] * inv_n);
+        };
+        if (KB == 1 && items <= kRows) {
+            // One item per lane of each warpgroup; the two warpgroups take
+            // alternate token parts and meet in shared memory.
+            const int e = quad * 32 + lane;
+            float s[8];
+            float* dst;
+            const bool head = region_sum(e, wg * parts, 2 * parts, s, dst);
+            if (wg == 1 && head) {
+                reinterpret_cast<float4*>(scratch + e * 8)[0] = make_float4(s[0], s[1], s[2], s[3]);
+                reinterpret_cast<float4*>(scratch + e * 8)[1] = make_float4(s[4], s[5], s[6], s[7]);
+            }
+            __syncthreads();
+            if (wg == 0 && head) {
+                const float4 u = reinterpret_cast<const float4*>(scratch + e * 8)[0];
+                const float4 w = reinterpret_cast<const float4*>(scratch + e * 8)[1];
+                s[0] += u.x; s[1] += u.y; s[2] += u.z; s[3] += u.w;
+                s[4] += w.x; s[5] += w.y; s[6] += w.z; s[7] += w.w;
+                store_mean(dst, s);
+            }
+        } else {
+            for (int e0 = warp * 32; e0 < items; e0 += kThreads) {
+                float s[8];
+                float* dst;
+                if (region_sum(e0 + lane, 0, parts, s, dst)) store_mean(dst, s);
             }
         }
     }
