@@ -110,6 +110,18 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// One region-sum item of a thread: 8 channels of one Q or K block of one
+// region of the tile, over the tokens first, first + stride, ...
+struct SumItem {
+    int pp;          // token part
+    int blk;         // staging block: 0..KB-1 Q, KB..2KB-1 K
+    int i, j;        // region column / row inside the tile
+    int ti, xi, t;   // first token: index in the region, column in the region, row in the tile
+    int o;           // 0: Q^r, 1: K^r
+    int dst_off;     // (head * R) * 32 + channel within the head
+    bool valid;      // e < items
+};
+
 struct TileCoord {
     int b, x0, y0;
 };
@@ -218,6 +230,36 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
         w_pending = true;
         for (int j = 0; j < kStages; ++j) issue_x(j);
     }
+    bool mma_pending = false;
+    // D = X_tile(j) W^T into TMEM; thread 0 only.  False if a wait gave up.
+    auto issue_mma = [&](uint32_t j) -> bool {
+        if (w_pending) {
+            if (!ptx::mbar_wait(wfull, 0, kWaitLimit)) return false;
+            w_pending = false;
+        }
+        const int stage = (int)(j % kStages);
+        if (!ptx::mbar_wait(afull + stage, (j / kStages) & 1u, kWaitLimit)) return false;
+        a_done = j + 1;
+        ptx::tc_fence_after();
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(kRows, kNChunk, false, false);
+        const uint32_t sAs = sA + stage * KB * kBlockBytes;
+#pragma unroll
+        for (int nb = 0; nb < 3 * C / kNChunk; ++nb)
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t a = ptx::smem_desc(sAs + kb * kBlockBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                    const uint64_t bd = ptx::smem_desc(sW + kb * 3 * C * 128 + nb * kNChunk * 128 + ks * 32, 16, 1024,
+                                                       ptx::kSwizzle128B);
+                    ptx::mma_bf16(tmem + nb * kNChunk, a, bd, idesc, (kb | ks) != 0);
+                }
+        ptx::mma_commit(mma_done);
+        mma_pending = true;
+        return true;
+    };
+    bool ok = true;
+    if (tid == 0 && blockIdx.x < p.tiles) ok = issue_mma(0);
 
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int row = tid & (kRows - 1);
@@ -225,44 +267,32 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
     const int parts = p.parts;
     const int pc = lane & 7;
     const int items = 8 * parts * 2 * KB * p.nrx * p.nry;
-    bool ok = true;
+    // Tile-invariant part of a region-sum item (see the region sums below).
+    auto make_item = [&](int e, int first) {
+        SumItem m;
+        m.pp = (e >> 3) % parts;
+        const int rest = (e >> 3) / parts;
+        m.blk = rest % (2 * KB);
+        const int reg = rest / (2 * KB);
+        m.j = reg / p.nrx;
+        m.i = reg - m.j * p.nrx;
+        m.valid = e < items;
+        m.ti = m.pp + first;
+        const int yi = m.ti / g.ws;
+        m.xi = m.ti - yi * g.ws;
+        m.t = (m.j * g.hs + yi) * p.bw + m.i * g.ws + m.xi;
+        m.o = m.blk / KB;
+        const int cin = (m.blk - m.o * KB) * 64 + pc * 8;
+        m.dst_off = (cin >> 5) * g.R * 32 + (cin & 31);
+        return m;
+    };
+    const SumItem split_item = make_item(quad * 32 + lane, wg * parts);
     uint32_t it = 0;
-    bool mma_pending = false;
 
     for (long long tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
         const TileCoord tc = tile_coord(tile, p);
-        const int stage = (int)(it % kStages);
 
-        // ---- D = X_tile W^T ----------------------------------------------------
-        if (tid == 0) {
-            bool got = true;
-            if (w_pending) {
-                got = ptx::mbar_wait(wfull, 0, kWaitLimit);
-                w_pending = !got;
-            }
-            if (got) got = ptx::mbar_wait(afull + stage, (it / kStages) & 1u, kWaitLimit);
-            if (got) {
-                a_done = it + 1;
-                ptx::tc_fence_after();
-                constexpr uint32_t idesc = ptx::idesc_bf16_f32(kRows, kNChunk, false, false);
-                const uint32_t sAs = sA + stage * KB * kBlockBytes;
-#pragma unroll
-                for (int nb = 0; nb < 3 * C / kNChunk; ++nb)
-#pragma unroll
-                    for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            const uint64_t a = ptx::smem_desc(sAs + kb * kBlockBytes + ks * 32, 16, 1024, ptx::kSwizzle128B);
-                            const uint64_t bd = ptx::smem_desc(sW + kb * 3 * C * 128 + nb * kNChunk * 128 + ks * 32, 16,
-                                                               1024, ptx::kSwizzle128B);
-                            ptx::mma_bf16(tmem + nb * kNChunk, a, bd, idesc, (kb | ks) != 0);
-                        }
-                ptx::mma_commit(mma_done);
-                mma_pending = true;
-            } else {
-                ok = false;
-            }
-        }
+        // ---- D = X_tile W^T was issued before the previous tile's region sums
         if (__syncthreads_or(!ok)) {
             ok = false;
             break;
@@ -318,6 +348,9 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
                 tma_store_4d(&tv, sOut + (2 * KB + kb) * kBlockBytes, kb * 64, tc.x0, tc.y0, tc.b);
             }
             bulk_commit();
+            // TMEM is free again (every row was read before the barrier): the
+            // next tile's MMAs run under this tile's region sums.
+            if (tile + gridDim.x < p.tiles) ok = issue_mma(it + 1);
         }
 
         // ---- region means of the staged Q and K ---------------------------------
@@ -328,19 +361,14 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
         // takes part; items past the end add zeros).  Eight consecutive lanes
         // read the eight chunks of one token row: conflict-free 16-byte loads.
         const int rx0 = tc.x0 / g.ws, ry0 = tc.y0 / g.hs;
-        auto region_sum = [&](int e, int first, int stride, float (&out)[8], float*& dst) -> bool {
-            const int pp = (e >> 3) % parts;
-            const int rest = (e >> 3) / parts;
-            const int blk = rest % (2 * KB), reg = rest / (2 * KB);
-            const int j = reg / p.nrx, i = reg - j * p.nrx;
-            const int rx = rx0 + i, ry = ry0 + j;
-            const bool live = e < items && rx < g.S && ry < g.S;
+        auto region_sum = [&](const SumItem& m, int stride, float (&out)[8], float*& dst) -> bool {
+            const int rx = rx0 + m.i, ry = ry0 + m.j;
+            const bool live = m.valid && rx < g.S && ry < g.S;
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-            int ti = pp + first;
+            int ti = m.ti;
             if (live && ti < g.n) {
-                const uint8_t* buf = smem + L::kOffOut + blk * kBlockBytes;  // blocks 0..KB-1: Q, then K
-                int yi = ti / g.ws, xi = ti - yi * g.ws;
-                int t = (j * g.hs + yi) * p.bw + i * g.ws + xi;
+                const uint8_t* buf = smem + L::kOffOut + m.blk * kBlockBytes;  // blocks 0..KB-1: Q, then K
+                int xi = m.xi, t = m.t;
                 for (; ti < g.n; ti += stride) {
                     const uint4 v = *reinterpret_cast<const uint4*>(buf + t * 128 + ((pc ^ (t & 7)) << 4));
                     acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
@@ -364,9 +392,8 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
             for (int off = 8; off < 8 * parts; off <<= 1)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) out[c] += __shfl_xor_sync(0xffffffffu, out[c], off);
-            const int o = blk / KB, cin = (blk - o * KB) * 64 + pc * 8;
-            dst = (o == 0 ? qr : kr) + (((size_t)tc.b * g.heads + (cin >> 5)) * g.R + ry * g.S + rx) * 32 + (cin & 31);
-            return live && pp == 0;
+            dst = (m.o == 0 ? qr : kr) + ((size_t)tc.b * g.heads * g.R + ry * g.S + rx) * 32 + m.dst_off;
+            return live && m.pp == 0;
         };
         auto store_mean = [&](float* dst, const float (&s)[8]) {
             reinterpret_cast<float4*>(dst)[0] = make_float4(s[0] * inv_n, s[1] * inv_n, s[2] * inv_n, s[3] * inv_n);
@@ -378,7 +405,7 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
             const int e = quad * 32 + lane;
             float s[8];
             float* dst;
-            const bool head = region_sum(e, wg * parts, 2 * parts, s, dst);
+            const bool head = region_sum(split_item, 2 * parts, s, dst);
             if (wg == 1 && head) {
                 reinterpret_cast<float4*>(scratch + e * 8)[0] = make_float4(s[0], s[1], s[2], s[3]);
                 reinterpret_cast<float4*>(scratch + e * 8)[1] = make_float4(s[4], s[5], s[6], s[7]);
@@ -395,7 +422,7 @@ bra_qkv_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ C
             for (int e0 = warp * 32; e0 < items; e0 += kThreads) {
                 float s[8];
                 float* dst;
-                if (region_sum(e0 + lane, 0, parts, s, dst)) store_mean(dst, s);
+                if (region_sum(make_item(e0 + lane, 0), parts, s, dst)) store_mean(dst, s);
             }
         }
     }
