@@ -210,7 +210,7 @@ def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return {"value": tokens / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    return {"value": tokens / el, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
             "sample": f"{calls} oracle calls of {bpc} of {shape.B} images ({tokens} tokens) "
                       f"in {el:.1f} s, float64, one thread"}
 
@@ -283,7 +283,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {**workload_config(shape, args.workload), "sample_images_per_step": bpc,
                    "local_context": bool(args.lce), "from_feature_map": bool(args.qkv)},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"{bpc} of {shape.B} images per step, float64 oracle, one thread"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
