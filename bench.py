@@ -27,6 +27,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -45,12 +46,13 @@ L2_BYTES = 126 * 2**20
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes per launch of the attention kernel on the stage-1 workload, from
-# an ncu capture, keyed by the sha256 of the kernel sources it was taken on;
-# reported as ``traffic`` only while the sources are unchanged.
+# an ncu capture, keyed by the sha256 of the kernel code it was taken on
+# (kernel_sources_hash: comments do not count); reported as ``traffic`` only
+# while that code is unchanged.
 TRAFFIC_RECORDS: dict[str, float] = {
     # ncu --set full capture of bra_attend_stack_kernel<4, 1, 0> on the stage-1 workload:
     # dram__bytes_read.sum 68.28 MB + dram__bytes_write.sum 4.28 MB
-    "87a9b4f22773ee876f8e80b8c22ff2de3a6ec63af952d6ca7be72c780640a920": 72.554752e6,
+    "de3711efbcd4ea77df2a9aba4a92dcb9d6452a8988dd0747246a23e183b13334": 72.554752e6,
 }
 
 
@@ -61,7 +63,7 @@ TRAFFIC_RECORDS: dict[str, float] = {
 QKV_TRAFFIC_RECORDS: dict[str, float] = {
     # ncu --set full capture of bra_qkv_kernel<1> (8 warps, next MMA under the region sums):
     # dram read 25.76 MB + write 20.27 MB
-    "a7357e391aff02e362258e5581ad4b65a7544619661754cd07013bdd5fd3a0a5": 46.031616e6,
+    "5474982f1906dccc5f9126cc3a60e458e6d92efc3665bffbef24bfaf1d6cbe60": 46.031616e6,
 }
 
 
@@ -123,15 +125,23 @@ def measured_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments or blank lines: edits to comments do not
+    change the code the counters were taken on."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_sources_hash(prefix: str = "attend") -> str:
-    """sha256 of the sources of the kernel named by ``prefix`` (its own files,
-    the TMA host code and the shared device headers)."""
+    """sha256 of the code (comments stripped) of the kernel named by
+    ``prefix``: its own files, the TMA host code and the shared device headers."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dynamic_sparse_attention_bra_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.startswith((prefix, "tma_host")) or name in ("common.cuh", "kernels.h", "tc_ptx.cuh"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()
 
 

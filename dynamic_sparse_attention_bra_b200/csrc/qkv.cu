@@ -14,11 +14,14 @@
 //     128-byte swizzled K-major layout the MMA reads; boxes that reach past
 //     the map are zero-filled on load and clipped on store.
 // Per tile, one elected thread issues D = X_tile W^T with M = 128, N = 192
-// per MMA, K = 16 per step, into TMEM; the 128 threads then read their row,
-// add the bias, round to bf16 into swizzled staging buffers (one per output
-// and 64-channel block), which TMA stores back; the same threads then sum the
-// staged Q and K columns of every region of the tile (deterministic, no
-// atomics: each region lies in exactly one tile) and write the means.
+// per MMA, K = 16 per step, into TMEM.  Two warpgroups share the 128 TMEM
+// lanes: each reads half of the output columns of its rows, adds the bias
+// and rounds to bf16 into swizzled staging buffers (one per output and
+// 64-channel block), which TMA stores back; then both sum the staged Q and K
+// columns of every region of the tile (deterministic, no atomics: each region
+// lies in exactly one tile) and write the means.  The next tile's MMAs are
+// issued as soon as this tile's rows have been read from TMEM, so they run
+// under the region sums.
 //
 // The weights (at most 96 KB) stay resident in shared memory for the CTA's
 // lifetime.  X tiles go through a ring of two buffers when C = 64 (one when
@@ -26,9 +29,11 @@
 // MMAs reading it have completed, so loads overlap the epilogue; two CTAs
 // share an SM when C = 64.
 //
-// Pooling reads the staging buffers with 16-byte loads: a thread sums one
+// Region sums read the staging buffers with 16-byte loads: a thread sums one
 // 8-channel chunk of one region over every parts-th token, and the parts
-// (lanes 8 apart) are folded with shuffles.
+// (lanes 8 apart) are folded with shuffles; when a tile has at most 128 sum
+// items the two warpgroups take alternate token parts and add their halves
+// through a small shared-memory scratch.
 #include "../../include/bra.h"
 #include "kernels.h"
 #include "qkv.h"
