@@ -8,6 +8,9 @@ synthetic inputs.  Prints one JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--lce] [--qkv]
 
+``--backward`` times bra_attend_backward (dQ, dK, dV for the routing of a
+forward pass made beforehand) on the same workload and reports its own line.
+
 ``--qkv`` starts every step from the feature map X instead of Q, K, V: the
 fused projection (Q, K, V and their region means in one kernel), routing on
 those means and attention (bra_forward_qkv), with seeded linear-layer
@@ -80,6 +83,8 @@ def parse(argv=None):
                    help="add the local context enhancement (bra_lce, seeded 5x5 depthwise weights) to every step")
     p.add_argument("--qkv", action="store_true",
                    help="start every step from the feature map: fused Q/K/V projection + routing + attention")
+    p.add_argument("--backward", action="store_true",
+                   help="time the attention gradients (bra_attend_backward) instead of the forward")
     return p.parse_args(argv)
 
 
@@ -498,10 +503,87 @@ def run_ours(args):
     return 0
 
 
+def run_backward(args):
+    """bra_attend_backward on one GPU: dQ, dK, dV (fp32) for a fixed routing."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--backward runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    shape, seed = bi.WORKLOADS[args.workload]
+    inp = bi.make_inputs(shape, seed)
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+    def dev_map(x):
+        t = torch.from_numpy(x)
+        return (t.view(torch.bfloat16) if shape.dtype == "bf16" else t).to(dev)
+
+    q, k, v = (dev_map(a) for a in (inp.q_store, inp.k_store, inp.v_store))
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device=dev)
+    idx = torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    g = torch.Generator().manual_seed(seed + 100)
+    go = torch.randn(q.shape, generator=g).to(tdt).to(dev)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    with torch.cuda.stream(stream):
+        bra.bra_forward(s, q, k, v, o, idx, ws, sp)  # the routing the gradients are taken for
+
+    def step():
+        bra.bra_attend_backward(s, q, k, v, idx, go, dq, dk, dv, ws, sp)
+
+    # Inputs and gradients (Q, K, V, dO read; dQ, dK, dV cleared and written in fp32)
+    # span more than the 126 MB L2 on the stage workloads.
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(args.steps):
+                step()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+    st = bra.bra_device_status(s, ws, sp)
+    if st != bra.BRA_OK:
+        raise RuntimeError(f"device status after timing: {bra.bra_status_string(st)}")
+    ms = start.elapsed_time(end) / args.steps
+    cnt = byte_counts(shape)
+    es = 2 if shape.dtype == "bf16" else 4
+    # minimal bytes: Q, K, V, dO and I^r read once, dQ, dK, dV written once in fp32
+    grad_bytes = 3 * shape.tokens * shape.C * 4
+    min_bytes = 4 * cnt["map"] + cnt["idx"] + grad_bytes
+    peak, peak_kind = measured_peaks()
+    achieved = min_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "BRA attention backward tokens/s on 1 B200", "value": shape.tokens / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype,
+        "data": "synthetic",
+        "config": {**workload_config(shape, args.workload), "gradients": "fp32", "element_bytes": es},
+        "roofline": {"kernel": "bra_attend_backward", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes": min_bytes, "launch_ms": ms},
+        "gpu_launches": args.steps,
+        "clocks": clocks.report(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.backward:
+        return run_backward(args)
     return run_ours(args)
 
 
