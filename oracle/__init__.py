@@ -80,7 +80,13 @@ def swapped_library(path: str):
 
 
 def _f64(x) -> np.ndarray:
-    return np.ascontiguousarray(x, dtype=np.float64)
+    """Contiguous float64 copy of an input; NaN and infinity are outside the
+    method's contract (the pages define the steps on real-valued maps), so they
+    are rejected rather than propagated."""
+    a = np.ascontiguousarray(x, dtype=np.float64)
+    if not np.isfinite(a).all():
+        raise ValueError("oracle inputs must be finite (NaN and infinity are outside the contract)")
+    return a
 
 
 def _ptr(a: np.ndarray, t):

@@ -368,3 +368,15 @@ def test_oracle_rejects_bad_shapes(bad):
     q = np.zeros((1, 8, 8, 8))
     with pytest.raises(ValueError):
         oracle.bra_forward(q, q, q, args["heads"], args["S"], args["topk"])
+
+
+@pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
+def test_non_finite_inputs_are_rejected(bad):
+    # Non-finite maps are outside the contract: the oracle refuses them instead
+    # of returning a result no reading of the pages defines.
+    q = np.random.default_rng(0).standard_normal((1, 4, 4, 4))
+    q[0, 1, 2, 3] = bad
+    with pytest.raises(ValueError):
+        oracle.region_pool(q, 1, 2)
+    with pytest.raises(ValueError):
+        oracle.qkv_projection(q, np.eye(4).repeat(3, axis=0))
