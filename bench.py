@@ -21,7 +21,8 @@ independent replica on its own batch (the path has no exchange step), and
 the value is all ranks' tokens over the slowest rank's device time.
 
 ``--impl reference`` times the float64 CPU oracle on bounded samples of the
-same workload (the comparison arm; rank 0 only).
+same workload, one image per host core per step (the comparison arm; rank 0
+only).
 """
 from __future__ import annotations
 
@@ -47,6 +48,7 @@ WORKLOAD = "stage1"
 METRIC = "BRA forward tokens/s on 1 B200 (bf16) and % of tensor/HBM roofline"
 L2_BYTES = 126 * 2**20
 FALLBACK_HBM_GBS = 6650.0
+DATASHEET_HBM_GBS = 7700.0  # B200 HGX nominal HBM3e bandwidth, for context beside the measured copy peak
 
 # DRAM bytes per launch of the attention kernel on the stage-1 workload, from
 # an ncu capture, keyed by the sha256 of the kernel code it was taken on
@@ -85,6 +87,8 @@ def parse(argv=None):
                    help="start every step from the feature map: fused Q/K/V projection + routing + attention")
     p.add_argument("--backward", action="store_true",
                    help="time the attention gradients (bra_attend_backward) instead of the forward")
+    p.add_argument("--per-workload", default="stage2,stage3,highres",
+                   help="other workloads timed in the same run (comma list; empty: none)")
     return p.parse_args(argv)
 
 
@@ -164,16 +168,33 @@ class ClockSampler:
         self.samples: list[int] = []
         self.reasons = 0
         self.max_mhz = None
+        self.matched_by = None
         self._stop = threading.Event()
         self._thread = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self._nvml = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._h, self.matched_by = self._handle(pynvml, device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:  # no NVML: report what we could not sample
             self._nvml = None
+
+    @staticmethod
+    def _handle(nv, device_index: int):
+        """NVML handle of the CUDA device ``device_index``.  NVML numbers the
+        GPUs of the machine and ignores CUDA_VISIBLE_DEVICES, so the device is
+        found by its UUID (else its PCI bus id), not by its CUDA index."""
+        import torch
+        props = torch.cuda.get_device_properties(device_index)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(f"GPU-{uuid}"), "uuid"
+            except Exception:
+                pass
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        return nv.nvmlDeviceGetHandleByPciBusId(bus), "pci_bus_id"
 
     def _run(self):
         nv = self._nvml
@@ -183,7 +204,7 @@ class ClockSampler:
                 self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
             except Exception:
                 return
-            time.sleep(0.002)
+            time.sleep(0.0002)
 
     def __enter__(self):
         if self._nvml is not None:
@@ -199,12 +220,83 @@ class ClockSampler:
     def report(self) -> dict:
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                "nvml_device_matched_by": self.matched_by}
+
+
+def host_cores() -> int:
+    """Cores this process may run on (the affinity mask, not the machine)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# State of one oracle worker process (filled by _oracle_worker_init).
+_WORKER: dict = {}
+
+
+def _oracle_worker_init(shape: bi.BraShape, seed: int, from_feature_map: bool, lce: bool) -> None:
+    import oracle
+    _WORKER["oracle"] = oracle
+    _WORKER["shape"] = shape
+    _WORKER["inp"] = bi.make_inputs(shape, seed)
+    _WORKER["proj"] = bi.make_projection_inputs(shape, seed) if from_feature_map else None
+    if lce:
+        rng = np.random.default_rng(seed + 77)
+        _WORKER["lce"] = (rng.standard_normal((shape.C, 5, 5)) / 5.0, rng.standard_normal(shape.C))
+    else:
+        _WORKER["lce"] = None
+
+
+def _oracle_image(i: int) -> int:
+    """The unmodified oracle's forward on image i of the batch (one thread);
+    returns the tokens processed."""
+    oracle, shape, inp, proj, lce = (_WORKER[k] for k in ("oracle", "shape", "inp", "proj", "lce"))
+    b = i % shape.B
+    sl = slice(b, b + 1)
+    if proj is not None:
+        q, k, v = oracle.qkv_projection(proj.x_f64[sl], proj.w_f64, proj.b_f64)
+    else:
+        q, k, v = inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl]
+    o, _ = oracle.bra_forward(q, k, v, shape.heads, shape.S, shape.topk)
+    if lce is not None:
+        o = o + oracle.local_context(v, lce[0], lce[1])
+    return shape.H * shape.W
+
+
+class OraclePool:
+    """``cores`` worker processes (spawned, so safe after CUDA is initialised),
+    each holding the seeded workload, running the oracle one image per task."""
+
+    def __init__(self, shape: bi.BraShape, seed: int, cores: int, from_feature_map: bool = False,
+                 lce: bool = False):
+        import multiprocessing as mp
+        self.cores = cores
+        self.pool = mp.get_context("spawn").Pool(cores, initializer=_oracle_worker_init,
+                                                 initargs=(shape, seed, from_feature_map, lce))
+        self.pool.map(_oracle_image, range(cores))  # inputs built, oracle loaded in every worker
+
+    def run(self, first_image: int, images: int) -> int:
+        return sum(self.pool.map(_oracle_image, range(first_image, first_image + images), chunksize=1))
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
 
 
 def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
-                          batches_per_call: int | None = None, from_feature_map: bool = False) -> dict:
-    """The float64 oracle (single thread) on bounded samples of the workload."""
+                          batches_per_call: int | None = None, from_feature_map: bool = False,
+                          all_cores: bool = True) -> dict:
+    """The float64 oracle on bounded samples of the workload: one thread, and
+    (``all_cores``) one worker process per host core, each running the
+    unmodified oracle on its own images."""
     import oracle
     inp = bi.make_inputs(shape, seed)
     proj = bi.make_projection_inputs(shape, seed) if from_feature_map else None
@@ -225,9 +317,25 @@ def cpu_oracle_throughput(shape: bi.BraShape, seed: int, budget_s: float = 10.0,
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return {"value": tokens / el, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{calls} oracle calls of {bpc} of {shape.B} images ({tokens} tokens) "
-                      f"in {el:.1f} s, float64, one thread"}
+    one = {"value": tokens / el, "unit": "tokens/s", "cores": 1, "host_cores": host_cores(), "kind": "oracle",
+           "sample": f"{calls} oracle calls of {bpc} of {shape.B} images ({tokens} tokens) "
+                     f"in {el:.1f} s, float64, one thread"}
+    cores = host_cores()
+    if not all_cores or cores <= 1:
+        return one
+    with OraclePool(shape, seed, cores, from_feature_map) as pool:
+        done = 0
+        t0 = time.perf_counter()
+        while True:
+            done += pool.run(done // (shape.H * shape.W), cores)
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+    images = done // (shape.H * shape.W)
+    return {"value": done / el, "unit": "tokens/s", "cores": cores, "host_cores": cores, "kind": "oracle",
+            "sample": f"{images} images of the {shape.B}-image batch ({done} tokens) in {el:.1f} s, float64, "
+                      f"one image per task on {cores} worker processes",
+            "single_thread": one}
 
 
 def max_over_ranks(values, world: int, device="cpu") -> list[float]:
@@ -259,51 +367,121 @@ def dist_env():
 
 
 def run_reference(args):
+    """The comparison arm: the float64 oracle, unmodified, on the host's cores.
+    Each step runs one image per core (a bounded sample of the batch), every
+    worker process running the oracle on its own image."""
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
     shape, seed = bi.WORKLOADS[args.workload]
-    import oracle
-    inp = bi.make_inputs(shape, seed)
-    proj = bi.make_projection_inputs(shape, seed) if args.qkv else None
-    bpc = 1  # one image per step: a bounded sample of the batch
-    lce_w = lce_b = None
-    if args.lce:
-        rng = np.random.default_rng(seed + 77)
-        lce_w = rng.standard_normal((shape.C, 5, 5)) / 5.0
-        lce_b = rng.standard_normal(shape.C)
-
-    def step(i):
-        sl = slice(i % shape.B, i % shape.B + bpc)
-        if args.qkv:
-            q, k, v = oracle.qkv_projection(proj.x_f64[sl], proj.w_f64, proj.b_f64)
-        else:
-            q, k, v = inp.q_f64[sl], inp.k_f64[sl], inp.v_f64[sl]
-        o, _ = oracle.bra_forward(q, k, v, shape.heads, shape.S, shape.topk)
-        if args.lce:
-            o = o + oracle.local_context(v, lce_w, lce_b)
-        return o
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(i)
-    el = time.perf_counter() - t0
-    tokens = args.steps * bpc * shape.H * shape.W
+    cores = host_cores()
+    with OraclePool(shape, seed, cores, from_feature_map=args.qkv, lce=args.lce) as pool:
+        for i in range(args.warmup):
+            pool.run(i * cores, cores)
+        tokens = 0
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            tokens += pool.run((args.warmup + i) * cores, cores)
+        el = time.perf_counter() - t0
     value = tokens / el
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**workload_config(shape, args.workload), "sample_images_per_step": bpc,
+        "config": {**workload_config(shape, args.workload), "sample_images_per_step": cores,
                    "local_context": bool(args.lce), "from_feature_map": bool(args.qkv)},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"{bpc} of {shape.B} images per step, float64 oracle, one thread"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "host_cores": cores, "kind": "oracle",
+                         "sample": f"{cores} of {shape.B} images per step, one per worker process, "
+                                   f"float64 oracle"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def measured_peak_tflops() -> float | None:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def roofline_time_s(shape: bi.BraShape, hbm_gbs: float, tflops: float | None) -> tuple[float, str]:
+    """The attention kernel's roofline time: the larger of its minimal bytes
+    over the HBM peak and its FLOPs over the bf16 tensor peak."""
+    t_hbm = byte_counts(shape)["attend"] / (hbm_gbs * 1e9)
+    t_tc = attention_flops(shape) / (tflops * 1e12) if tflops else 0.0
+    return (t_tc, "tensor") if t_tc > t_hbm else (t_hbm, "hbm")
+
+
+def time_workload(name: str, steps: int, warmup: int, dev, stream) -> dict:
+    """Step time (bra_forward back to back) and the attention kernel's own
+    launch time (events around each bra_attend) on another workload, with
+    rotating input sets larger than L2, in the same process as the headline."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape, seed = bi.WORKLOADS[name]
+    inp = bi.make_inputs(shape, seed)
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    cnt = byte_counts(shape)
+    set_bytes = 4 * cnt["map"] + cnt["idx"]
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    base = [torch.from_numpy(a).view(tdt) if shape.dtype == "bf16" else torch.from_numpy(a)
+            for a in (inp.q_store, inp.k_store, inp.v_store)]
+    sets = []
+    for _ in range(nsets):
+        q, k, v = (t.to(dev) for t in base)
+        sets.append(dict(q=q, k=k, v=v, o=torch.empty_like(q),
+                         idx=torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device=dev),
+                         ws=torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device=dev)))
+    sp = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            b = sets[i % nsets]
+            bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with ClockSampler(dev.index) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(steps):
+                b = sets[i % nsets]
+                bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+            end.record(stream)
+            for i in range(steps):
+                b = sets[i % nsets]
+                bra.bra_route(s, b["q"], b["k"], b["idx"], b["ws"], sp)
+                ev[i][0].record(stream)
+                bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    for b in sets:
+        st = bra.bra_device_status(s, b["ws"], sp)
+        if st != bra.BRA_OK:
+            raise RuntimeError(f"{name}: device status after timing: {bra.bra_status_string(st)}")
+    step_ms = start.elapsed_time(end) / steps
+    attend_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    peak, peak_kind = measured_peaks()
+    t_roof, bound = roofline_time_s(shape, peak, measured_peak_tflops())
+    del sets
+    torch.cuda.empty_cache()
+    return {
+        "workload": workload_config(shape, name)["workload"], "tokens_per_step": shape.tokens,
+        "step_ms": step_ms, "tokens_per_s": shape.tokens / (step_ms * 1e-3),
+        "attend": {"launch_ms": attend_ms, "bound": bound, "roofline_us": t_roof * 1e6,
+                   "frac": t_roof / (attend_ms * 1e-3),
+                   "achieved_gbs": cnt["attend"] / (attend_ms * 1e-3) / 1e9,
+                   "achieved_tflops": attention_flops(shape) / (attend_ms * 1e-3) / 1e12,
+                   "algorithmic_bytes": cnt["attend"], "flops": attention_flops(shape),
+                   "peak_kind": peak_kind},
+        "path_frac": cnt["path_min"] / (peak * 1e9) / (step_ms * 1e-3),
+        "steps": steps, "l2": f"rotating {nsets} input sets ({nsets * set_bytes / 2**20:.0f} MiB)",
+        "clocks": clocks.report(),
+    }
 
 
 def run_ours(args):
@@ -453,6 +631,12 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
 
     total_ms, attend_ms, e2e_ms, qkv_ms = max_over_ranks([total_ms, attend_ms, e2e_ms, qkv_ms], world, dev)
+
+    # The other workloads' attention and step times, on one GPU (same process).
+    per_workload = {}
+    if world == 1 and not args.qkv and not args.lce:
+        for name in [w for w in args.per_workload.split(",") if w and w != args.workload]:
+            per_workload[name] = time_workload(name, args.steps, max(args.warmup, 3), dev, stream)
     ms_per_step = total_ms / args.steps
     tokens = shape.tokens * world
     value = whole_job_tokens_per_s(shape.tokens, world, ms_per_step)
@@ -475,6 +659,7 @@ def run_ours(args):
                 "kernel": "bra_attend", "bound": "hbm", "achieved": achieved, "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                 "algorithmic_bytes": cnt["attend"], "launch_ms": attend_ms,
+                "datasheet_peak": DATASHEET_HBM_GBS, "frac_of_datasheet": achieved / DATASHEET_HBM_GBS,
             },
             "path_roofline": {
                 "min_bytes": cnt[path_key], "flops": attention_flops(shape),
@@ -486,6 +671,8 @@ def run_ours(args):
             "gpu_launches": (4 if args.lce else 3) * args.steps,
             "clocks": clocks.report(),
         }
+        if per_workload:
+            line["per_workload"] = per_workload
         if args.qkv:
             qkv_gbs = cnt["qkv"] / (qkv_ms * 1e-3) / 1e9
             line["qkv_roofline"] = {

@@ -3,20 +3,19 @@
 // in a caller-supplied workspace, for callers that cannot allocate device
 // memory themselves.  It runs the same pool and route kernels as bra_route.
 //
-// Set-up: the first call on each device looks up that device's address of
-// the array with cudaGetSymbolAddress (the device must be current, which it
-// is for the caller's stream) and caches it; later calls reuse it.  That
-// first call should come before any stream capture.  The array's name in
-// host code is only a host-side handle, never a device address, so kernels
-// are always given the looked-up pointer.
+// Set-up: every call looks up the current device's address of the array
+// with cudaGetSymbolAddress (which allocates nothing; the device must be
+// current, which it is for the caller's stream), so the address is never
+// stale, even after a device reset has reloaded the library's module.  The
+// first call on a device may load the module, so it should come before any
+// stream capture.  The array's name in host code is only a host-side handle,
+// never a device address, so kernels are always given the looked-up pointer.
 //
 // Every call on a device shares the one array and leaves the last call's
 // means in it; nothing in it needs to start at zero (the pool kernel writes
 // every mean the route kernel reads).  Calls that overlap on the GPU (two
 // streams, or two host threads) race on the array.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "../../include/bra.h"
 #include "common.cuh"
@@ -29,21 +28,11 @@ namespace {
 constexpr size_t kNoAllocMeans = BRA_NOALLOC_MAX_MEANS;
 static __device__ __align__(256) float g_route_scratch[2 * kNoAllocMeans];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-float* g_scratch_ptr[kMaxDevices] = {};
-
 // Device address of g_route_scratch on the current device, or nullptr.
 float* scratch_for_current_device() {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev] = static_cast<float*>(p);
-    }
-    return g_scratch_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
+    return static_cast<float*>(p);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

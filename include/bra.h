@@ -168,9 +168,11 @@ bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stre
  * GPU that loads the library holds it, 2 * BRA_NOALLOC_MAX_MEANS floats =
  * 8 MiB, until the process exits).  Limit: B * heads * S*S * d must not
  * exceed BRA_NOALLOC_MAX_MEANS, else BRA_ERR_UNSUPPORTED (and nothing is
- * launched); other argument errors are those of bra_route.  The first call
- * on a device looks up the array's device address there (the caller's
- * current device); make that first call before any stream capture.  All
+ * launched); other argument errors are those of bra_route.  Every call
+ * looks up the array's device address on the caller's current device (so a
+ * device reset does not leave a stale address behind); the first call on a
+ * device may load the library's module there, so make that first call
+ * before any stream capture.  All
  * calls share the array, so calls that overlap on the GPU race: order them
  * (e.g. one stream).  Allocates nothing, host or device.
  */

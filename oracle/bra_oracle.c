@@ -27,13 +27,15 @@
  *   5. gather the K/V tokens of the k routed regions and run token-to-token
  *      softmax attention over their union (section 2.2 step 4).
  *
- * Readings where the pages are silent (each listed in the design notes):
+ * Readings where the pages are silent:
  *   - heads: C = heads * d, every head is routed and attended on its own
  *     (channels [h*d, (h+1)*d));
  *   - the softmax logits are scaled by 1/sqrt(d); A^r is not scaled;
  *   - region order and token order inside a region are row-major;
  *   - top-k ties go to the lower region index, and each I^r row lists its
  *     regions by (affinity descending, index ascending);
+ *   - attention runs over the union of the routed tokens: a caller-given
+ *     I^r row that lists a region twice attends to its tokens once;
  *   - the local-context term (section 2.2 step 4, third bullet, and the
  *     "+ dwconv(value)" of pseudocode step 7) is a separate function,
  *     oracle_local_context: a 5x5 depthwise filter over the H x W map with
@@ -152,7 +154,7 @@ int oracle_token_attention(const double* q, const double* k, const double* v,
                            const int32_t* idx, double* o)
 {
     if (check_shape(B, H, W, C, heads, S, topk)) return ORACLE_EINVAL;
-    int R = S * S, d = C / heads, n = (H / S) * (W / S), kn = topk * n;
+    int R = S * S, d = C / heads, n = (H / S) * (W / S), kn = topk * n;  /* kn: most keys a query can have */
     double scale = 1.0 / sqrt((double)d);
     double* s = (double*)malloc(sizeof(double) * (size_t)kn);
     size_t* key_off = (size_t*)malloc(sizeof(size_t) * (size_t)kn);
@@ -162,14 +164,21 @@ int oracle_token_attention(const double* q, const double* k, const double* v,
         for (int h = 0; h < heads && !rc; ++h)
             for (int r = 0; r < R && !rc; ++r) {
                 const int32_t* route = idx + (((size_t)b * heads + h) * R + r) * topk;
-                /* gather: offsets of the routed key/value tokens */
+                /* gather: offsets of the routed key/value tokens.  The query
+                 * attends over the union of its routed tokens, so a region
+                 * listed more than once contributes its tokens once (its
+                 * first listing); top-k never lists a region twice. */
+                int nkeys = 0;
                 for (int m = 0; m < topk; ++m) {
                     int rr = route[m];
                     if (rr < 0 || rr >= R) { rc = ORACLE_EINVAL; break; }
+                    int listed_before = 0;
+                    for (int mm = 0; mm < m; ++mm) listed_before |= route[mm] == rr;
+                    if (listed_before) continue;
                     for (int t = 0; t < n; ++t) {
                         int y, x;
                         region_token(H, W, S, rr, t, &y, &x);
-                        key_off[m * n + t] = (((size_t)b * H + y) * W + x) * C + (size_t)h * d;
+                        key_off[nkeys++] = (((size_t)b * H + y) * W + x) * C + (size_t)h * d;
                     }
                 }
                 if (rc) break;
@@ -178,20 +187,20 @@ int oracle_token_attention(const double* q, const double* k, const double* v,
                     region_token(H, W, S, r, t, &y, &x);
                     size_t qoff = (((size_t)b * H + y) * W + x) * C + (size_t)h * d;
                     double mx = -INFINITY;
-                    for (int j = 0; j < kn; ++j) {
+                    for (int j = 0; j < nkeys; ++j) {
                         double dot = 0.0;
                         for (int c = 0; c < d; ++c) dot += q[qoff + c] * k[key_off[j] + c];
                         s[j] = dot * scale;
                         if (s[j] > mx) mx = s[j];
                     }
                     double den = 0.0;
-                    for (int j = 0; j < kn; ++j) {
+                    for (int j = 0; j < nkeys; ++j) {
                         s[j] = exp(s[j] - mx);
                         den += s[j];
                     }
                     for (int c = 0; c < d; ++c) {
                         double num = 0.0;
-                        for (int j = 0; j < kn; ++j) num += s[j] * v[key_off[j] + c];
+                        for (int j = 0; j < nkeys; ++j) num += s[j] * v[key_off[j] + c];
                         o[qoff + c] = num / den;
                     }
                 }

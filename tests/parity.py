@@ -27,6 +27,15 @@ import numpy as np
 REL_GAP = 1e-4
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 
+# (case, max-abs error, tolerance, ambiguous routing rows, routing rows) of
+# every GPU parity comparison in this process, printed at the end of the
+# pytest run (tests/conftest.py) so the margin to the tolerance is on record.
+MARGINS: list[tuple[str, float, float, int, int]] = []
+
+
+def record_margin(case: str, err: float, tol: float, ambiguous: int = 0, rows: int = 0) -> None:
+    MARGINS.append((case, float(err), float(tol), int(ambiguous), int(rows)))
+
 
 @dataclasses.dataclass
 class RouteReport:

@@ -17,7 +17,7 @@ import pytest
 
 import bra_inputs as bi
 import oracle
-from parity import TOL, compare_routes
+from parity import TOL, compare_routes, record_margin
 
 pytestmark = pytest.mark.gpu
 
@@ -121,7 +121,8 @@ def test_forward_from_feature_map(name):
     rep = compare_routes(out["idx"], oracle.region_affinity(qr, kr))
     assert not rep.mismatches, rep.mismatches[:5]
     o_ref = oracle.token_attention(q, k, v, out["idx"], sh.heads, sh.S)
-    err = np.abs(out["o"] - o_ref).max()
+    err = float(np.abs(out["o"] - o_ref).max())
+    record_margin(f"forward_qkv {name}", err, TOL["bf16"], rep.ambiguous, rep.rows)
     assert err <= TOL["bf16"], err
 
 

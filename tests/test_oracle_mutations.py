@@ -24,6 +24,7 @@ MUTATIONS = [
     ("softmax_weights_perturbed", "s[j] = exp(s[j] - mx);", "s[j] = exp(s[j] - mx + 1e-3 * j);"),
     ("values_from_keys", "num += s[j] * v[key_off[j] + c];", "num += s[j] * k[key_off[j] + c];"),
     ("first_route_only", "int rr = route[m];", "int rr = route[0];"),
+    ("repeats_counted_twice", "                    if (listed_before) continue;\n", ""),
 ]
 
 
@@ -52,6 +53,7 @@ def test_pins_catch_mutation(tmp_path, name, old, new):
         pins.test_worked_example_by_hand,
         pins.test_region_permutation_equivariance,
         lambda: pins.test_brute_force_tiny(2, 2),
+        lambda: pins.test_repeated_routes_attend_the_union(1),
     ]
     failures = 0
     with oracle.swapped_library(lib):

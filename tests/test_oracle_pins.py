@@ -199,6 +199,32 @@ def test_gather_equals_region_masked_dense(cfg):
     np.testing.assert_allclose(o, dense_attention(q, kk, v, heads, mask), rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("heads", [1, 2])
+def test_repeated_routes_attend_the_union(heads):
+    """A caller-given routing may list a region more than once; the query
+    attends over the union of its routed tokens (each token once), which is
+    the region-masked dense formulation with the mask built from the set of
+    listed regions."""
+    B, H, W, C, S, k = 1, 8, 8, 8, 4, 3
+    q, kk, v = qkv(B, H, W, C, S, 35 + heads)
+    rng = np.random.default_rng(heads)
+    idx = rng.integers(0, S * S, size=(B, heads, S * S, k)).astype(np.int32)
+    idx[0, 0, :4] = [[2, 2, 2], [5, 1, 5], [0, 0, 7], [9, 3, 3]]
+    o = oracle.token_attention(q, kk, v, idx, heads, S)
+    reg = bi.region_map(H, W, S).reshape(-1)
+    routed = np.zeros((B, heads, S * S, S * S), dtype=bool)
+    for m in range(k):
+        np.put_along_axis(routed, idx[..., m:m + 1].astype(np.int64), True, axis=-1)
+    mask = routed[:, :, reg][:, :, :, reg]
+    np.testing.assert_allclose(o, dense_attention(q, kk, v, heads, mask), rtol=0, atol=1e-12)
+    # a region listed three times gives what the same region listed once gives
+    once = np.ascontiguousarray(idx[..., :1])  # row 0 of head 0 is [2]
+    o1 = oracle.token_attention(q, kk, v, once, heads, S)
+    d = C // heads
+    in_region0 = (reg == 0).reshape(H, W)
+    assert np.array_equal(o[0][in_region0][:, :d], o1[0][in_region0][:, :d])
+
+
 def test_constant_values_give_constant_output():
     """softmax weights sum to one: V = c everywhere gives O = c."""
     B, H, W, C, heads, S, k = 1, 8, 8, 8, 2, 4, 2
