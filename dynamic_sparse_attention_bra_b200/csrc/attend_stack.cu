@@ -55,7 +55,7 @@ namespace {
 
 constexpr int kMaxSlots = 4;    // 64 rows / 16 tokens
 constexpr int kMaxRoutes = 16;  // kn <= 256 with n >= 16
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kMaxSBuf = 8;
 constexpr uint32_t kWait = 1u << 22;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -80,7 +80,8 @@ struct StackPlan {
     uint32_t stage_bytes;   // Q (2 x 64 rows) + K + V of one tile
     uint32_t k_off, v_off;  // offsets inside a stage
     uint32_t p_half;        // one half of a P buffer: ceil(N / 64) atoms of 64 rows x 128 B
-    uint32_t p_off;         // offset of the P buffers
+    int pin;                // 1: a tile's P is written over its own stage's Q and K (dead once S is done)
+    uint32_t p_off;         // offset of the separate P buffers (pin == 0)
     uint32_t ones_off;      // offset of a bf16 ones tile [16][N] (row sums of P by MMA)
     uint32_t bar_off;       // offset of barriers and tile metadata
     uint32_t smem_bytes;    // dynamic shared memory requested (incl. alignment slack)
@@ -378,7 +379,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 if (!wait_or_abort(&sb->p_full[pb], (i / p.np) & 1, sb, status)) break;
                 ptx::tc_fence_after();
                 const uint32_t stage = sbase + (uint32_t)s * p.stage_bytes;
-                const uint32_t pbase = sbase + p.p_off + (uint32_t)pb * 2u * p.p_half;
+                const uint32_t pbase = p.pin ? stage : sbase + p.p_off + (uint32_t)pb * 2u * p.p_half;
                 if constexpr (CP) {
                     // One accumulator per (half, region g) over g's kn-key window, the
                     // O blocks 48 columns apart; steps of all accumulators interleaved.
@@ -492,7 +493,8 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             const bool all_live = live == full_live;
             if (slot_ok) {
                 const uint32_t col0 = sbuf * p.N + slot * p.kn;
-                const uint32_t prow = sbase + p.p_off + (uint32_t)pb * 2u * p.p_half + half * p.p_half + m * 128;
+                const uint32_t pbuf = p.pin ? sbase + (uint32_t)s * p.stage_bytes : sbase + p.p_off + (uint32_t)pb * 2u * p.p_half;
+                const uint32_t prow = pbuf + half * p.p_half + m * 128;
                 // 16 p values of window columns c .. c + 15 as 8 bf16 pairs: two
                 // 16-byte chunks of the row's 128-byte swizzled atom line.
                 auto write_p16 = [&](int c, const uint32_t* packed) {
@@ -625,6 +627,10 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     // on a barrier's parity need the barrier's previous phase complete: a
     // group's earlier tiles must cover the tile `stages` (and `nsb`) before,
     // so groups <= stages and nsb a multiple of the groups.
+    // P goes over its own stage's Q and K once S = Q K^T is done reading them,
+    // when it fits there and needs no zero fill (a block-diagonal P is zero
+    // outside each row's window, which separate buffers keep from the start).
+    p->pin = (p->cp || p->Gq == 1) && 2u * p->p_half <= p->v_off ? 1 : 0;
     static const int kOptions[6][3] = {{4, 1, 5}, {2, 2, 3}, {2, 1, 3}, {1, 2, 3}, {2, 1, 2}, {1, 1, 2}};
     int stages = 0;
     bool found = false;
@@ -633,7 +639,8 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
         p->wgs = kOptions[o][0];
         p->pdepth = kOptions[o][1];
         p->np = p->wgs * p->pdepth;
-        const uint32_t used = 1024 + misc + ones_bytes + (uint32_t)p->np * 2u * p->p_half;
+        const uint32_t pbytes = p->pin ? 0u : (uint32_t)p->np * 2u * p->p_half;
+        const uint32_t used = 1024 + misc + ones_bytes + pbytes;
         stages = used < kSmemBudget ? (int)((kSmemBudget - used) / p->stage_bytes) : 0;
         found = stages >= kOptions[o][2] && stages >= p->wgs;
     }
@@ -641,7 +648,7 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     if (stages > kMaxStages) stages = kMaxStages;
     p->stages = stages;
     p->p_off = (uint32_t)stages * p->stage_bytes;
-    p->ones_off = p->p_off + (uint32_t)p->np * 2u * p->p_half;
+    p->ones_off = p->p_off + (p->pin ? 0u : (uint32_t)p->np * 2u * p->p_half);
     p->bar_off = p->ones_off + ones_bytes;
     p->smem_bytes = p->bar_off + (uint32_t)sizeof(Barriers) + 1024;
     p->nprod = stages < kProd ? stages : kProd;
