@@ -635,7 +635,10 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     int stages = 0;
     bool found = false;
     for (int o = 0; o < 6 && !found; ++o) {
-        if (kOptions[o][0] > max_groups || p->nsb % kOptions[o][0] != 0) continue;
+        // a group holds one S buffer per tile whose epilogue is pending
+        if (kOptions[o][0] > max_groups || p->nsb % kOptions[o][0] != 0 ||
+            p->nsb < kOptions[o][0] * kOptions[o][1])
+            continue;
         p->wgs = kOptions[o][0];
         p->pdepth = kOptions[o][1];
         p->np = p->wgs * p->pdepth;

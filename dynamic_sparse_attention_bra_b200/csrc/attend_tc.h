@@ -19,4 +19,19 @@ bra_status attend_tc_launch(const Geometry& g, const void* q, const void* k, con
 bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* idx, void* o, int* status, cudaStream_t stream);
 
+// Persistent variant for maps of at most 256 tokens (BiFormer stage 3): each
+// (batch, head) slice's Q, K, V in shared memory, S dense over the slice,
+// each query's softmax masked to its routed regions' keys.
+bool attend_slice_covers(const Geometry& g);
+bra_status attend_slice_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* idx, void* o, int* status, cudaStream_t stream);
+
+// Warp-level MMA variant for small regions (n % 16 == 0, topk * n of 32, 64
+// or 128) whose (batch, head) K and V slices fit twice in an SM's shared
+// memory (BiFormer stage 2): one CTA per slice, routed rows gathered by
+// per-lane operand addresses.
+bool attend_warp_covers(const Geometry& g);
+bra_status attend_warp_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                              const int32_t* idx, void* o, int* status, cudaStream_t stream);
+
 }  // namespace bra

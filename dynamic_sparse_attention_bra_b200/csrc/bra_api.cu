@@ -69,16 +69,24 @@ Workspace carve(const Geometry& g, void* ws) {
 }
 
 // Attention kernel selection.  The environment variable BRA_ATTEND_KERNEL
-// (read on every call) pins one kernel for testing: "stack" (persistent
-// tcgen05, regions of 16..64 tokens), "tiled" (tcgen05 per 128-query tile),
-// "simt" (CUDA cores); a pinned kernel that does not cover the shape makes
-// the call return BRA_ERR_UNSUPPORTED.  Unset or "auto": the first of those
-// that covers the shape (tensor-core kernels for bf16 only).
-enum class AttendKernel { kAuto, kStack, kTiled, kSimt };
+// (read on every call) pins one kernel for testing: "slice" (persistent
+// tcgen05, a map of at most 256 tokens per (batch, head), dense with a
+// routing mask), "warp" (warp-level MMAs over a (batch, head) slice's K and V
+// resident in shared memory, small regions), "stack" (persistent tcgen05,
+// regions of 16..64 tokens), "tiled" (tcgen05 per 128-query tile), "simt" (CUDA cores); a
+// pinned kernel that does not cover the shape makes the call return
+// BRA_ERR_UNSUPPORTED.  Unset or "auto": the slice kernel for small maps,
+// else the warp kernel when it covers the shape and each query region routes
+// to several regions (a gather per query tile would re-read K and V topk
+// times), else the first of stack, tiled, simt that covers it (tensor-core
+// kernels for bf16 only).
+enum class AttendKernel { kAuto, kSlice, kWarp, kStack, kTiled, kSimt };
 
 AttendKernel attend_kernel_choice() {
     const char* e = getenv("BRA_ATTEND_KERNEL");
     if (!e) return AttendKernel::kAuto;
+    if (!strcmp(e, "slice")) return AttendKernel::kSlice;
+    if (!strcmp(e, "warp")) return AttendKernel::kWarp;
     if (!strcmp(e, "stack")) return AttendKernel::kStack;
     if (!strcmp(e, "tiled")) return AttendKernel::kTiled;
     if (!strcmp(e, "simt")) return AttendKernel::kSimt;
@@ -100,6 +108,17 @@ bra_status attend_impl(const bra_shape* s, const Geometry& g, const void* q, con
     if (g.B == 0) return BRA_OK;
     const bool bf16 = s->dtype == BRA_DTYPE_BF16;
     const AttendKernel choice = attend_kernel_choice();
+    if (bf16 && (choice == AttendKernel::kSlice || (choice == AttendKernel::kAuto && attend_slice_covers(g)))) {
+        const bra_status rc = attend_slice_launch(g, q, k, v, idx, o, w.status, st);
+        if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kSlice) return rc;
+    }
+    if (choice == AttendKernel::kSlice) return BRA_ERR_UNSUPPORTED;
+    if (bf16 && (choice == AttendKernel::kWarp ||
+                 (choice == AttendKernel::kAuto && g.topk > 1 && attend_warp_covers(g)))) {
+        const bra_status rc = attend_warp_launch(g, q, k, v, idx, o, w.status, st);
+        if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kWarp) return rc;
+    }
+    if (choice == AttendKernel::kWarp) return BRA_ERR_UNSUPPORTED;
     if (bf16 && (choice == AttendKernel::kAuto || choice == AttendKernel::kStack)) {
         const bra_status rc = attend_stack_launch(g, q, k, v, idx, o, w.status, st);
         if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kStack) return rc;
@@ -201,10 +220,9 @@ bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void
     if (cudaMemsetAsync(dq, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess ||
         cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
         return BRA_ERR_CUDA;
-    return launch_attend_backward(shape->dtype == BRA_DTYPE_BF16, q, k, v, idx, grad_o, dq, dk, dv, g,
-                                  carve(g, workspace).status, st) == cudaSuccess
-               ? BRA_OK
-               : BRA_ERR_CUDA;
+    const cudaError_t e = launch_attend_backward(shape->dtype == BRA_DTYPE_BF16, q, k, v, idx, grad_o, dq, dk, dv, g,
+                                                 carve(g, workspace).status, st);
+    return e == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
 }
 
 bra_status bra_qkv_project(const bra_shape* shape, const void* x, const void* w_qkv, const float* b_qkv, void* q,

@@ -50,7 +50,8 @@ def pinned_kernel(request, monkeypatch):
 
 # Every attention kernel on every shape it covers (the default run above uses
 # the first kernel that covers each shape).
-KERNEL_CASES = [(k, w) for k in ("stack", "tiled", "simt") for w in ("stage1", "stage2", "stage3", "highres")]
+KERNEL_CASES = [(k, w) for k in ("slice", "warp", "stack", "tiled", "simt")
+                for w in ("stage1", "stage2", "stage3", "highres")]
 
 
 @pytest.mark.parametrize("pinned_kernel,name", KERNEL_CASES, indirect=["pinned_kernel"],
@@ -64,6 +65,7 @@ def test_each_kernel_on_workloads(pinned_kernel, name):
         if e.status != bra.BRA_ERR_UNSUPPORTED:
             raise
         assert pinned_kernel != "simt"
+        assert (pinned_kernel, name) not in (("warp", "stage2"), ("slice", "stage3"))
         pytest.skip(f"{pinned_kernel} does not cover {name}")
 
 
@@ -240,3 +242,115 @@ def test_workspace_reused_across_calls():
         torch.cuda.synchronize()
         assert torch.equal(idx, idx2)
         assert torch.equal(o.view(torch.int16), o2.view(torch.int16))
+
+
+# The resident-slice warp kernel on the shapes it covers: several routes of
+# 16 or 32 tokens, 64 and 128 keys per query region, one image, many slices.
+WARP_CASES = {
+    "stage2_batch8": (8, 28, 28, 128, 4, 7, 4),
+    "stage2_one_image": (1, 28, 28, 128, 4, 7, 4),      # 4 slices: most CTAs idle
+    "topk8_128_keys": (4, 28, 28, 128, 4, 7, 8),        # two query regions per half
+    "regions_of_32": (4, 32, 16, 64, 2, 4, 2),          # 8 x 4 regions, R = 16
+    "odd_heads": (3, 28, 28, 96, 3, 7, 4),
+    "many_slices": (150, 28, 28, 32, 1, 7, 4),          # 150 slices: two for some CTAs
+}
+
+
+@pytest.mark.parametrize("kernel", ["warp"])
+@pytest.mark.parametrize("name", list(WARP_CASES))
+def test_warp_kernel(name, kernel, monkeypatch):
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", kernel)
+    B, H, W, C, heads, S, topk = WARP_CASES[name]
+    check_case(bi.BraShape(B, H, W, C, heads, S, topk, "bf16"), 200 + len(name), label=f"{name} [{kernel}]")
+
+
+def attend_given_routes(shape, seed, idx):
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    inp = bi.make_inputs(shape, seed)
+    q, k, v = device_inputs(inp)
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device="cuda")
+    o = torch.zeros_like(q)
+    bra.bra_attend(s, q, k, v, torch.from_numpy(idx).cuda(), o, ws)
+    status = bra.bra_device_status(s, ws)
+    return inp, o.float().cpu().numpy(), status
+
+
+@pytest.mark.parametrize("kernel", ["warp"])
+def test_warp_repeated_routes_attend_the_union(kernel, monkeypatch):
+    import dynamic_sparse_attention_bra_b200 as bra
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", kernel)
+    shape = bi.BraShape(2, 28, 28, 64, 2, 7, 4, "bf16")
+    rng = np.random.default_rng(5)
+    idx = rng.integers(0, shape.R, size=(shape.B, shape.heads, shape.R, shape.topk)).astype(np.int32)
+    idx[0, 0, :3] = [[3, 3, 3, 3], [7, 1, 7, 2], [0, 0, 48, 48]]
+    inp, o, status = attend_given_routes(shape, 13, idx)
+    assert status == bra.BRA_OK
+    ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx, shape.heads, shape.S)
+    err = float(np.abs(o - ref).max())
+    record_margin(f"repeated_routes [{kernel}]", err, TOL["bf16"])
+    assert err <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("kernel", ["warp"])
+@pytest.mark.parametrize("bad_value", [-1, 49, 1 << 30])
+def test_warp_bad_route_is_reported_not_read(bad_value, kernel, monkeypatch):
+    import dynamic_sparse_attention_bra_b200 as bra
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", kernel)
+    shape = bi.BraShape(1, 28, 28, 64, 2, 7, 4, "bf16")
+    idx = np.tile(np.arange(4, dtype=np.int32), (1, 2, 49, 1))
+    idx[0, 1, 20, 2] = bad_value
+    inp, o, status = attend_given_routes(shape, 4, idx)
+    assert status == bra.BRA_ERR_BAD_ROUTE
+    # every other region is still attended correctly
+    ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, np.where(idx < 0, 0, np.minimum(idx, 48)),
+                                 shape.heads, shape.S)
+    reg = bi.region_map(shape.H, shape.W, shape.S)
+    keep = np.ones(o.shape, dtype=bool)
+    keep[0][reg == 20, 32:64] = False
+    assert np.abs(o - ref)[keep].max() <= TOL["bf16"]
+
+
+# The dense-slice kernel on the maps it covers (at most 256 tokens per
+# (batch, head)): one and two 128-query units per slice, regions of one to
+# sixteen tokens, routes up to S^2, bad and repeated routes.
+SLICE_CASES = {
+    "stage3_batch8": (8, 14, 14, 256, 8, 7, 16),
+    "stage4_full": (8, 7, 7, 512, 16, 7, 49),           # one-token regions, k = S^2
+    "map_16x12": (3, 16, 12, 64, 2, 4, 3),              # 192 tokens, 4 x 3 regions
+    "map_12x10": (5, 12, 10, 96, 3, 2, 1),              # 120 tokens: one unit, 6 x 5 regions
+    "one_region": (2, 8, 8, 64, 2, 1, 1),               # S = 1: dense attention
+    "many_slices": (40, 14, 14, 256, 8, 7, 4),          # 320 slices
+}
+
+
+@pytest.mark.parametrize("name", list(SLICE_CASES))
+def test_slice_kernel(name, monkeypatch):
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", "slice")
+    B, H, W, C, heads, S, topk = SLICE_CASES[name]
+    check_case(bi.BraShape(B, H, W, C, heads, S, topk, "bf16"), 300 + len(name), label=f"{name} [slice]")
+
+
+def test_slice_repeated_and_bad_routes(monkeypatch):
+    import dynamic_sparse_attention_bra_b200 as bra
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", "slice")
+    shape = bi.BraShape(2, 14, 14, 64, 2, 7, 5, "bf16")
+    rng = np.random.default_rng(8)
+    idx = rng.integers(0, shape.R, size=(shape.B, shape.heads, shape.R, shape.topk)).astype(np.int32)
+    idx[0, 0, :3] = [[3, 3, 3, 3, 3], [7, 1, 7, 2, 1], [0, 0, 48, 48, 9]]
+    inp, o, status = attend_given_routes(shape, 17, idx)
+    assert status == bra.BRA_OK
+    ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx, shape.heads, shape.S)
+    err = float(np.abs(o - ref).max())
+    record_margin("repeated_routes [slice]", err, TOL["bf16"])
+    assert err <= TOL["bf16"]
+    bad = idx.copy()
+    bad[1, 1, 30, 4] = 49
+    inp, o, status = attend_given_routes(shape, 17, bad)
+    assert status == bra.BRA_ERR_BAD_ROUTE
+    reg = bi.region_map(shape.H, shape.W, shape.S)
+    skipped = np.zeros(o.shape, dtype=bool)
+    skipped[1][reg == 30, 32:64] = True
+    assert (o[skipped] == 0).all()  # the region's outputs are left as they were
+    assert np.abs(o - ref)[~skipped & (np.arange(shape.B) == 1)[:, None, None, None]].max() <= TOL["bf16"]
