@@ -444,6 +444,7 @@ def time_workload(name: str, steps: int, warmup: int, dev, stream) -> dict:
             bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     with ClockSampler(dev.index) as clocks:
         with torch.cuda.stream(stream):
@@ -458,13 +459,19 @@ def time_workload(name: str, steps: int, warmup: int, dev, stream) -> dict:
                 ev[i][0].record(stream)
                 bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
                 ev[i][1].record(stream)
+            a0.record(stream)
+            for i in range(steps):
+                b = sets[i % nsets]
+                bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
+            a1.record(stream)
         torch.cuda.synchronize(dev)
     for b in sets:
         st = bra.bra_device_status(s, b["ws"], sp)
         if st != bra.BRA_OK:
             raise RuntimeError(f"{name}: device status after timing: {bra.bra_status_string(st)}")
     step_ms = start.elapsed_time(end) / steps
-    attend_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    attend_iso_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    attend_ms = a0.elapsed_time(a1) / steps
     peak, peak_kind = measured_peaks()
     t_roof, bound = roofline_time_s(shape, peak, measured_peak_tflops())
     del sets
@@ -474,6 +481,7 @@ def time_workload(name: str, steps: int, warmup: int, dev, stream) -> dict:
         "step_ms": step_ms, "tokens_per_s": shape.tokens / (step_ms * 1e-3),
         "attend": {"launch_ms": attend_ms, "bound": bound, "roofline_us": t_roof * 1e6,
                    "frac": t_roof / (attend_ms * 1e-3),
+                   "launch_ms_isolated": attend_iso_ms, "frac_isolated": t_roof / (attend_iso_ms * 1e-3),
                    "achieved_gbs": cnt["attend"] / (attend_ms * 1e-3) / 1e9,
                    "achieved_tflops": attention_flops(shape) / (attend_ms * 1e-3) / 1e12,
                    "algorithmic_bytes": cnt["attend"], "flops": attention_flops(shape),
@@ -555,14 +563,18 @@ def run_ours(args):
     # Timed region: K steps of the public forward call back to back (pooling,
     # routing and attention per step, chained by programmatic dependent
     # launch), events only at its two ends.  A second pass over the same K
-    # steps brackets each attention launch with events on the same stream for
-    # the attention kernel's own average duration (an event between two
-    # launches ends their overlap, so this pass is not the step time).
+    # steps brackets each attention launch with events on the same stream
+    # (``launch_ms_isolated``: each launch alone, its set-up and pipeline fill
+    # exposed; an event between two launches ends their overlap, so this pass
+    # is not the step time), then times K attention launches back to back
+    # (``launch_ms``: the kernel's average launch period, as in a stream of
+    # attention calls).
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     ev_qkv = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)] if args.qkv else []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         if world > 1:
             torch.distributed.barrier()
@@ -587,11 +599,19 @@ def run_ours(args):
                 ev[i][0].record(stream)
                 bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
                 ev[i][1].record(stream)
+            # the attention kernel alone, K launches back to back on the routes of
+            # the pass above: its average launch period
+            a0.record(stream)
+            for i in range(args.steps):
+                b = sets[i % nsets]
+                bra.bra_attend(s, b["q"], b["k"], b["v"], b["idx"], b["o"], b["ws"], sp)
+            a1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     total_ms = start.elapsed_time(end)
-    attend_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    attend_iso_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    attend_ms = a0.elapsed_time(a1) / args.steps
     qkv_ms = sum(a.elapsed_time(b) for a, b in ev_qkv) / args.steps if args.qkv else 0.0
     for b in sets:
         st = bra.bra_device_status(s, b["ws"], sp)
@@ -630,7 +650,8 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
 
-    total_ms, attend_ms, e2e_ms, qkv_ms = max_over_ranks([total_ms, attend_ms, e2e_ms, qkv_ms], world, dev)
+    total_ms, attend_ms, attend_iso_ms, e2e_ms, qkv_ms = max_over_ranks(
+        [total_ms, attend_ms, attend_iso_ms, e2e_ms, qkv_ms], world, dev)
 
     # The other workloads' attention and step times, on one GPU (same process).
     per_workload = {}
@@ -659,6 +680,9 @@ def run_ours(args):
                 "kernel": "bra_attend", "bound": "hbm", "achieved": achieved, "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                 "algorithmic_bytes": cnt["attend"], "launch_ms": attend_ms,
+                "launch_timing": "CUDA events around K attention launches back to back (average period)",
+                "launch_ms_isolated": attend_iso_ms,
+                "frac_isolated": cnt["attend"] / (attend_iso_ms * 1e-3) / 1e9 / peak,
                 "datasheet_peak": DATASHEET_HBM_GBS, "frac_of_datasheet": achieved / DATASHEET_HBM_GBS,
             },
             "path_roofline": {

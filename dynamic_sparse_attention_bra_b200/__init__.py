@@ -30,9 +30,13 @@ __all__ = [
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libbra_b200.so")
+# BRA_LIBRARY selects another build of the same library, e.g. the debug build
+# libbra_b200_debug.so (output-index checks in the attention kernels).
+library_path = os.environ.get("BRA_LIBRARY") or os.path.join(_HERE, "libbra_b200.so")
+debug_library_path = os.path.join(_HERE, "libbra_b200_debug.so")
 
-BRA_OK, BRA_ERR_INVALID_ARG, BRA_ERR_UNSUPPORTED, BRA_ERR_CUDA, BRA_ERR_TIMEOUT, BRA_ERR_BAD_ROUTE = range(6)
+(BRA_OK, BRA_ERR_INVALID_ARG, BRA_ERR_UNSUPPORTED, BRA_ERR_CUDA, BRA_ERR_TIMEOUT, BRA_ERR_BAD_ROUTE,
+ BRA_ERR_BOUNDS) = range(7)
 BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",

@@ -40,27 +40,33 @@ def deps() -> list[str]:
                               + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+DEBUG_LIB = os.path.join(HERE, "libbra_b200_debug.so")
+
+
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile (if stale) and return the library path."""
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-o", tmp, *sources()]
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, debug: bool = False) -> str:
+    """Compile (if stale) and return the library path.  ``debug``: the
+    -DBRA_DEBUG build (output-index checks in the attention kernels) as
+    libbra_b200_debug.so, for tests."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    flags = [*NVCC_FLAGS, *(extra or []), *(["-DBRA_DEBUG"] if debug else [])]
+    cmd = [nvcc(), *flags, "-I", INCLUDE, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True,
+                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None, debug="--debug" in sys.argv))

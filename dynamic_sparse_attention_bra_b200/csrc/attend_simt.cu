@@ -133,8 +133,10 @@ bra_attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     if (active && sub == 0) {
         const float inv = 1.f / l;
         T* out = o + qoff;
+        if (in_bounds(qoff + D - 1, map_elems(g), status)) {
 #pragma unroll
-        for (int c = 0; c < D; ++c) out[c] = from_f32<T>(acc[c] * inv);
+            for (int c = 0; c < D; ++c) out[c] = from_f32<T>(acc[c] * inv);
+        }
     }
 }
 

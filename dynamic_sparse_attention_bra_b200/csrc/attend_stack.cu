@@ -451,15 +451,15 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             const float l = __uint_as_float(lw);
             const bool write = st.region >= 0 && l > 0.f;
             const float inv = write ? 1.f / l : 0.f;
-            int4* dst = write ? reinterpret_cast<int4*>(o + token_offset(g, st.b, st.region, tok) + (size_t)st.h * 32)
-                              : nullptr;
+            const size_t ooff = write ? token_offset(g, st.b, st.region, tok) + (size_t)st.h * 32 : 0;
+            int4* dst = write && in_bounds(ooff + 31, map_elems(g), status) ? reinterpret_cast<int4*>(o + ooff) : nullptr;
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
                 if (h16 == 1 && slot_ok) {
                     ptx::tmem_ld16(tmem + lane_addr + o_col + 16, r);
                     ptx::tmem_wait16(r);
                 }
-                if (write) {
+                if (dst) {
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         uint32_t w[4];

@@ -379,9 +379,10 @@ bra_attend_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             tok = tok0 + row;
         }
         const float inv = 1.f / l_run;
-        uint4* dst = reinterpret_cast<uint4*>(o + token_offset(g, b, reg, tok) + (size_t)h * 32);
+        const size_t ooff = token_offset(g, b, reg, tok) + (size_t)h * 32;
+        uint4* dst = reinterpret_cast<uint4*>(o + ooff);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 4 && in_bounds(ooff + 31, map_elems(g), status); ++c) {
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {

@@ -218,6 +218,7 @@ bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_cons
         }
         // O rows gq and gq + 8: channels 8n + 2tq, 8n + 2tq + 1
         const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+        if (!in_bounds((orow0 > orow1 ? orow0 : orow1) + 31, map_elems(g), status)) continue;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
             const int c = 8 * n + 2 * tq;

@@ -285,6 +285,7 @@ bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stre
     if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return BRA_ERR_CUDA;
     if (host == kDevTimeout) return BRA_ERR_TIMEOUT;
     if (host == kDevBadRoute) return BRA_ERR_BAD_ROUTE;
+    if (host == kDevBounds) return BRA_ERR_BOUNDS;
     return host == 0 ? BRA_OK : BRA_ERR_CUDA;
 }
 
@@ -296,6 +297,7 @@ const char* bra_status_string(bra_status status) {
         case BRA_ERR_CUDA: return "CUDA error";
         case BRA_ERR_TIMEOUT: return "device-side wait timed out";
         case BRA_ERR_BAD_ROUTE: return "routing index out of range";
+        case BRA_ERR_BOUNDS: return "index outside its buffer (debug build)";
     }
     return "unknown status";
 }

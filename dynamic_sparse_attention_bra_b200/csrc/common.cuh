@@ -20,10 +20,33 @@ struct Geometry {
 };
 
 // Status words at the start of the workspace status block.
-enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 4, kDevBadRoute = 5 };
+enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 4, kDevBadRoute = 5, kDevBounds = 6 };
 
 __device__ __forceinline__ void raise_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
+}
+
+// Index checks of a debug build (compiled with -DBRA_DEBUG): an access whose
+// last element ``last`` is not below ``count`` elements of its buffer is
+// recorded as kDevBounds in the status block and skipped.  A normal build
+// compiles the checks away (the function returns true).
+__device__ __forceinline__ bool in_bounds(size_t last, size_t count, int* status) {
+#ifdef BRA_DEBUG
+    if (last >= count) {
+        raise_status(status, kDevBounds);
+        return false;
+    }
+#else
+    (void)last;
+    (void)count;
+    (void)status;
+#endif
+    return true;
+}
+
+// Elements of a [B, H, W, C] map.
+__host__ __device__ __forceinline__ size_t map_elems(const Geometry& g) {
+    return (size_t)g.B * g.H * g.W * g.C;
 }
 
 // Element loads/stores widened to fp32.

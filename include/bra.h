@@ -60,7 +60,9 @@ typedef enum {
     BRA_ERR_UNSUPPORTED = 2, /* valid BRA problem this build does not cover */
     BRA_ERR_CUDA = 3,        /* a CUDA call or a kernel launch failed       */
     BRA_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out          */
-    BRA_ERR_BAD_ROUTE = 5    /* bra_attend saw a routing index outside [0, S*S) */
+    BRA_ERR_BAD_ROUTE = 5,   /* bra_attend saw a routing index outside [0, S*S) */
+    BRA_ERR_BOUNDS = 6       /* debug build only: a kernel caught an output index
+                                outside its buffer and skipped the access      */
 } bra_status;
 
 typedef enum { BRA_DTYPE_F32 = 0, BRA_DTYPE_BF16 = 1 } bra_dtype;
@@ -153,7 +155,9 @@ bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, c
 /*
  * Reads (synchronising ``stream``) and clears the device status block in
  * ``workspace``: BRA_OK, BRA_ERR_TIMEOUT (a bounded wait in a kernel gave up;
- * that kernel's outputs are incomplete) or BRA_ERR_BAD_ROUTE.
+ * that kernel's outputs are incomplete), BRA_ERR_BAD_ROUTE or, in a library
+ * built with -DBRA_DEBUG (libbra_b200_debug.so, which checks the output index
+ * of every attention-kernel store against its buffer), BRA_ERR_BOUNDS.
  */
 bra_status bra_device_status(const bra_shape* shape, void* workspace, void* stream);
 

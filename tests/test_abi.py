@@ -35,10 +35,18 @@ def test_library_exports_every_declared_symbol():
     assert set(bra.EXPORTED_SYMBOLS) <= set(declared_functions())
 
 
+def test_debug_build_exports_the_same_symbols():
+    """The -DBRA_DEBUG build (output-index checks) is a drop-in for the library."""
+    lib = ctypes.CDLL(bra.debug_library_path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
 def test_version_and_strings():
     assert bra._lib.bra_version() >= 100
     assert bra.bra_status_string(0) == "ok"
     assert "range" in bra.bra_status_string(5)
+    assert "debug" in bra.bra_status_string(bra.BRA_ERR_BOUNDS)
 
 
 S1 = dict(B=64, H=56, W=56, C=64, heads=2, S=7, topk=1, dtype="bf16")
