@@ -50,15 +50,27 @@ L2_BYTES = 126 * 2**20
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 7700.0  # B200 HGX nominal HBM3e bandwidth, for context beside the measured copy peak
 
-# DRAM bytes per launch of the attention kernel on the stage-1 workload, from
-# an ncu capture, keyed by the sha256 of the kernel code it was taken on
-# (kernel_sources_hash: comments do not count); reported as ``traffic`` only
-# while that code is unchanged.
-TRAFFIC_RECORDS: dict[str, float] = {
-    # ncu --set full capture of bra_attend_stack_kernel<4, 1, 0> on the stage-1 workload:
-    # dram__bytes_read.sum 68.28 MB + dram__bytes_write.sum 4.28 MB
-    "de3711efbcd4ea77df2a9aba4a92dcb9d6452a8988dd0747246a23e183b13334": 72.554752e6,
+# DRAM bytes per launch of each workload's attention kernel, from one ncu
+# capture, keyed by the sha256 of that kernel's code (kernel_file_hash:
+# comments do not count); reported as ``traffic`` only while the code is
+# unchanged.  With topk = 1 (stage 1) unrouted K and V regions are never read
+# and O is still dirty in L2 when the launch ends, so the figure is below the
+# algorithmic bytes.
+TRAFFIC_RECORDS: dict[str, dict[str, float]] = {
+    # ncu --set full, bra_attend_stack_kernel<4, 1, 0>, stage 1: read 68.26 MB + write 3.83 MB
+    "attend_stack.cu": {"37bdbeac0461348046559275bff62cf569565ddf91474f947747f0c6fcb8d94f": 72.095744e6},
+    # ncu --set full, bra_attend_warp_kernel<64> (12 warps), stage 2: read 38.77 MB + write 0.06 MB
+    "attend_warp.cu": {"0d86e7003b2f7dcb5aef6e442dbeee5b83f879c4e62fdc3e26bd769a7cb8bc58": 38.835456e6},
+    # ncu --set full, bra_attend_flash_kernel, highres: read 12.64 MB + write 0 MB
+    "attend_flash.cu": {"d6305cc7bc804bc43de0a31e74b516fa158d686d14c1ddd9034c4c964b32d6d7": 12.64e6},
+    # ncu --set full, bra_attend_slice_kernel, stage 3: read 20.95 MB + write 0 MB
+    "attend_slice.cu": {"eac7cbf607005191d84ac43bf035f66cdc772598a208926b8674cd8b4c51028e": 20.947968e6},
 }
+
+# The file holding each workload's attention kernel (the kernel bra_attend
+# chooses for that shape).
+KERNEL_FILE = {"stage1": "attend_stack.cu", "stage2": "attend_warp.cu", "stage3": "attend_slice.cu",
+               "highres": "attend_flash.cu", "detection": "attend_stack.cu", "tiny": "attend_simt.cu"}
 
 
 # DRAM bytes per launch of the fused projection kernel on the stage-1 workload
@@ -88,7 +100,7 @@ def parse(argv=None):
     p.add_argument("--backward", action="store_true",
                    help="time the attention gradients (bra_attend_backward) instead of the forward")
     p.add_argument("--per-workload", default="stage2,stage3,highres",
-                   help="other workloads timed in the same run (comma list; empty: none)")
+                   help="other workloads timed in the same run (comma list; 'none': none)")
     return p.parse_args(argv)
 
 
@@ -140,6 +152,24 @@ def _code_only(text: str) -> str:
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
     return "\n".join(ln for ln in lines if ln)
+
+
+def kernel_file_hash(name: str) -> str:
+    """sha256 of the code (comments stripped) of one kernel file and the shared
+    device headers and TMA host code it builds on."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dynamic_sparse_attention_bra_b200", "csrc")
+    for f in [name, "common.cuh", "kernels.h", "tc_ptx.cuh", "tma_host.cu", "tma_host.h"]:
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str) -> float | None:
+    """ncu DRAM bytes per launch of the workload's attention kernel, if the
+    kernel's code is the one they were taken on."""
+    name = KERNEL_FILE.get(workload)
+    return TRAFFIC_RECORDS.get(name, {}).get(kernel_file_hash(name)) if name else None
 
 
 def kernel_sources_hash(prefix: str = "attend") -> str:
@@ -485,7 +515,8 @@ def time_workload(name: str, steps: int, warmup: int, dev, stream) -> dict:
                    "achieved_gbs": cnt["attend"] / (attend_ms * 1e-3) / 1e9,
                    "achieved_tflops": attention_flops(shape) / (attend_ms * 1e-3) / 1e12,
                    "algorithmic_bytes": cnt["attend"], "flops": attention_flops(shape),
-                   "peak_kind": peak_kind},
+                   "peak_kind": peak_kind, "kernel_file": KERNEL_FILE.get(name),
+                   "traffic": recorded_traffic(name)},
         "path_frac": cnt["path_min"] / (peak * 1e9) / (step_ms * 1e-3),
         "steps": steps, "l2": f"rotating {nsets} input sets ({nsets * set_bytes / 2**20:.0f} MiB)",
         "clocks": clocks.report(),
@@ -656,7 +687,7 @@ def run_ours(args):
     # The other workloads' attention and step times, on one GPU (same process).
     per_workload = {}
     if world == 1 and not args.qkv and not args.lce:
-        for name in [w for w in args.per_workload.split(",") if w and w != args.workload]:
+        for name in [w for w in args.per_workload.split(",") if w in bi.WORKLOADS and w != args.workload]:
             per_workload[name] = time_workload(name, args.steps, max(args.warmup, 3), dev, stream)
     ms_per_step = total_ms / args.steps
     tokens = shape.tokens * world
@@ -666,8 +697,7 @@ def run_ours(args):
         peak, peak_kind = measured_peaks()
         achieved = cnt["attend"] / (attend_ms * 1e-3) / 1e9
         path_key = "path_min_qkv" if args.qkv else "path_min"
-        digest = kernel_sources_hash()
-        traffic = TRAFFIC_RECORDS.get(digest)
+        traffic = recorded_traffic(args.workload)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -34,4 +34,11 @@ bool attend_warp_covers(const Geometry& g);
 bra_status attend_warp_launch(const Geometry& g, const void* q, const void* k, const void* v,
                               const int32_t* idx, void* o, int* status, cudaStream_t stream);
 
+// Persistent flash-style variant for regions of a multiple of 128 tokens
+// (the dense-prediction map): 128-query tiles, keys streamed in blocks of 128
+// with a running maximum, output accumulated in registers.
+bool attend_flash_covers(const Geometry& g);
+bra_status attend_flash_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* idx, void* o, int* status, cudaStream_t stream);
+
 }  // namespace bra

@@ -19,7 +19,7 @@
 // registers) and O written once.  Two CTAs share an SM, so one's slice load
 // overlaps the other's arithmetic.
 //
-// Work: one CTA per slice (grid = B * heads); 8 warps take the slice's
+// Work: one CTA per slice (grid = B * heads); 12 warps take the slice's
 // (region, 16-query chunk) items in turn.  The slice's K and V arrive as one
 // 4-D TMA box per region each (64-byte rows, 64-byte swizzle, region r at
 // byte r * n * 64), completion on one mbarrier (bounded wait; on expiry the
@@ -37,7 +37,7 @@
 namespace bra {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 12;
 constexpr int kThreads = 32 * kWarps;
 constexpr uint32_t kWait = 1u << 22;
 constexpr float kLog2e = 1.4426950408889634f;

@@ -72,21 +72,23 @@ Workspace carve(const Geometry& g, void* ws) {
 // (read on every call) pins one kernel for testing: "slice" (persistent
 // tcgen05, a map of at most 256 tokens per (batch, head), dense with a
 // routing mask), "warp" (warp-level MMAs over a (batch, head) slice's K and V
-// resident in shared memory, small regions), "stack" (persistent tcgen05,
-// regions of 16..64 tokens), "tiled" (tcgen05 per 128-query tile), "simt" (CUDA cores); a
+// resident in shared memory, small regions), "flash" (persistent tcgen05,
+// regions of a multiple of 128 tokens, keys streamed in blocks with a running
+// maximum), "stack" (persistent tcgen05, regions of 16..64 tokens), "tiled" (tcgen05 per 128-query tile), "simt" (CUDA cores); a
 // pinned kernel that does not cover the shape makes the call return
 // BRA_ERR_UNSUPPORTED.  Unset or "auto": the slice kernel for small maps,
 // else the warp kernel when it covers the shape and each query region routes
 // to several regions (a gather per query tile would re-read K and V topk
-// times), else the first of stack, tiled, simt that covers it (tensor-core
-// kernels for bf16 only).
-enum class AttendKernel { kAuto, kSlice, kWarp, kStack, kTiled, kSimt };
+// times), else the first of flash, stack, tiled, simt that covers it
+// (tensor-core kernels for bf16 only).
+enum class AttendKernel { kAuto, kSlice, kWarp, kFlash, kStack, kTiled, kSimt };
 
 AttendKernel attend_kernel_choice() {
     const char* e = getenv("BRA_ATTEND_KERNEL");
     if (!e) return AttendKernel::kAuto;
     if (!strcmp(e, "slice")) return AttendKernel::kSlice;
     if (!strcmp(e, "warp")) return AttendKernel::kWarp;
+    if (!strcmp(e, "flash")) return AttendKernel::kFlash;
     if (!strcmp(e, "stack")) return AttendKernel::kStack;
     if (!strcmp(e, "tiled")) return AttendKernel::kTiled;
     if (!strcmp(e, "simt")) return AttendKernel::kSimt;
@@ -119,6 +121,11 @@ bra_status attend_impl(const bra_shape* s, const Geometry& g, const void* q, con
         if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kWarp) return rc;
     }
     if (choice == AttendKernel::kWarp) return BRA_ERR_UNSUPPORTED;
+    if (bf16 && (choice == AttendKernel::kFlash || (choice == AttendKernel::kAuto && attend_flash_covers(g)))) {
+        const bra_status rc = attend_flash_launch(g, q, k, v, idx, o, w.status, st);
+        if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kFlash) return rc;
+    }
+    if (choice == AttendKernel::kFlash) return BRA_ERR_UNSUPPORTED;
     if (bf16 && (choice == AttendKernel::kAuto || choice == AttendKernel::kStack)) {
         const bra_status rc = attend_stack_launch(g, q, k, v, idx, o, w.status, st);
         if (rc != BRA_ERR_UNSUPPORTED || choice == AttendKernel::kStack) return rc;

@@ -41,6 +41,7 @@ def bands_intact(buf) -> bool:
 KERNEL_SHAPES = [
     ("slice", (2, 14, 14, 256, 8, 7, 16)),
     ("warp", (2, 28, 28, 128, 4, 7, 4)),
+    ("flash", (1, 64, 64, 64, 2, 4, 2)),
     ("stack", (2, 56, 56, 64, 2, 7, 1)),
     ("tiled", (1, 32, 32, 64, 2, 2, 2)),
     ("simt", (1, 16, 16, 64, 2, 4, 3)),

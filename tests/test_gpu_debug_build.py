@@ -27,6 +27,7 @@ cases = [
     ("slice", (2, 14, 14, 256, 8, 7, 16, "bf16")),
     ("warp", (2, 28, 28, 128, 4, 7, 4, "bf16")),
     ("warp", (3, 28, 28, 96, 3, 7, 4, "bf16")),
+    ("flash", (1, 64, 64, 64, 2, 4, 2, "bf16")),
     ("stack", (4, 56, 56, 64, 2, 7, 1, "bf16")),
     ("stack", (2, 28, 28, 128, 4, 7, 4, "bf16")),
     ("tiled", (1, 32, 32, 64, 2, 2, 2, "bf16")),
@@ -46,4 +47,4 @@ def test_debug_build_reports_no_out_of_bounds_index():
     env = dict(os.environ, BRA_LIBRARY=lib)
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
-    assert r.stdout.count(" ok ") == 8, r.stdout
+    assert r.stdout.count(" ok ") == 9, r.stdout

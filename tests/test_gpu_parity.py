@@ -50,7 +50,7 @@ def pinned_kernel(request, monkeypatch):
 
 # Every attention kernel on every shape it covers (the default run above uses
 # the first kernel that covers each shape).
-KERNEL_CASES = [(k, w) for k in ("slice", "warp", "stack", "tiled", "simt")
+KERNEL_CASES = [(k, w) for k in ("slice", "warp", "flash", "stack", "tiled", "simt")
                 for w in ("stage1", "stage2", "stage3", "highres")]
 
 
@@ -65,7 +65,7 @@ def test_each_kernel_on_workloads(pinned_kernel, name):
         if e.status != bra.BRA_ERR_UNSUPPORTED:
             raise
         assert pinned_kernel != "simt"
-        assert (pinned_kernel, name) not in (("warp", "stage2"), ("slice", "stage3"))
+        assert (pinned_kernel, name) not in (("warp", "stage2"), ("slice", "stage3"), ("flash", "highres"))
         pytest.skip(f"{pinned_kernel} does not cover {name}")
 
 
@@ -354,3 +354,46 @@ def test_slice_repeated_and_bad_routes(monkeypatch):
     skipped[1][reg == 30, 32:64] = True
     assert (o[skipped] == 0).all()  # the region's outputs are left as they were
     assert np.abs(o - ref)[~skipped & (np.arange(shape.B) == 1)[:, None, None, None]].max() <= TOL["bf16"]
+
+
+# The flash kernel on the shapes it covers (regions of a multiple of 128
+# tokens): 256- and 128-token regions, two and eight key blocks per tile,
+# one route, k = S^2, an odd number of tiles per CTA.
+FLASH_CASES = {
+    "highres_b1": (1, 128, 128, 64, 2, 8, 4),
+    "regions_128": (2, 64, 32, 64, 2, 4, 3),          # 16 x 8 regions: one block per route
+    "one_route": (2, 64, 64, 64, 2, 4, 1),
+    "dense_k": (1, 32, 64, 64, 2, 2, 4),              # 16 x 32 regions, k = S^2
+    "odd_tiles": (1, 64, 64, 96, 3, 4, 2),            # 3 heads: tiles not a multiple of the grid
+}
+
+
+@pytest.mark.parametrize("name", list(FLASH_CASES))
+def test_flash_kernel(name, monkeypatch):
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", "flash")
+    B, H, W, C, heads, S, topk = FLASH_CASES[name]
+    check_case(bi.BraShape(B, H, W, C, heads, S, topk, "bf16"), 400 + len(name), label=f"{name} [flash]")
+
+
+def test_flash_repeated_and_bad_routes(monkeypatch):
+    import dynamic_sparse_attention_bra_b200 as bra
+    monkeypatch.setenv("BRA_ATTEND_KERNEL", "flash")
+    shape = bi.BraShape(1, 64, 64, 64, 2, 4, 3, "bf16")
+    rng = np.random.default_rng(9)
+    idx = rng.integers(0, shape.R, size=(shape.B, shape.heads, shape.R, shape.topk)).astype(np.int32)
+    idx[0, 0, :3] = [[3, 3, 3], [7, 1, 7], [0, 15, 15]]
+    inp, o, status = attend_given_routes(shape, 19, idx)
+    assert status == bra.BRA_OK
+    ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx, shape.heads, shape.S)
+    err = float(np.abs(o - ref).max())
+    record_margin("repeated_routes [flash]", err, TOL["bf16"])
+    assert err <= TOL["bf16"]
+    bad = idx.copy()
+    bad[0, 1, 5, 2] = -3
+    inp, o, status = attend_given_routes(shape, 19, bad)
+    assert status == bra.BRA_ERR_BAD_ROUTE
+    reg = bi.region_map(shape.H, shape.W, shape.S)
+    skipped = np.zeros(o.shape, dtype=bool)
+    skipped[0][reg == 5, 32:64] = True
+    assert (o[skipped] == 0).all()
+    assert np.abs(o - ref)[~skipped].max() <= TOL["bf16"]
