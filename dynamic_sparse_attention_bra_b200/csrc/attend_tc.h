@@ -27,9 +27,10 @@ bra_status attend_slice_launch(const Geometry& g, const void* q, const void* k, 
                                const int32_t* idx, void* o, int* status, cudaStream_t stream);
 
 // Warp-level MMA variant for small regions (n % 16 == 0, topk * n of 32, 64
-// or 128) whose (batch, head) K and V slices fit twice in an SM's shared
-// memory (BiFormer stage 2): one CTA per slice, routed rows gathered by
-// per-lane operand addresses.
+// or 128, maps of at most 256 x 256) whose (batch, head) K and V slices fit
+// twice in an SM's shared memory (BiFormer stage 2): persistent, one CTA per
+// SM over an equal share of the items, slices double-buffered, routed rows
+// gathered by per-lane operand addresses.
 bool attend_warp_covers(const Geometry& g);
 bra_status attend_warp_launch(const Geometry& g, const void* q, const void* k, const void* v,
                               const int32_t* idx, void* o, int* status, cudaStream_t stream);

@@ -15,17 +15,21 @@
 // 16-query chunk of a region, reads the routed regions' K and V rows in place
 // from the resident slice, keeps S, the softmax and P in registers (the
 // accumulator layout of S is the operand layout of P), and writes O.  Each
-// slice's K and V cross the load path once; Q is read once (straight into
-// registers) and O written once.  Two CTAs share an SM, so one's slice load
-// overlaps the other's arithmetic.
+// slice's K and V cross the load path once per CTA that works on it; Q is
+// read once (straight into registers) and O written once.
 //
-// Work: one CTA per slice (grid = B * heads); 12 warps take the slice's
-// (region, 16-query chunk) items in turn.  The slice's K and V arrive as one
-// 4-D TMA box per region each (64-byte rows, 64-byte swizzle, region r at
-// byte r * n * 64), completion on one mbarrier (bounded wait; on expiry the
-// CTA records kDevTimeout and writes nothing).  Routes: a region listed more
-// than once counts once (later listings are masked), and a query region with
-// an out-of-range route is reported (BRA_ERR_BAD_ROUTE) and not written.
+// Work: persistent, one CTA per SM.  All (slice, region, 16-query chunk)
+// items are split into equal contiguous ranges, one per CTA (a CTA's range
+// spans two or three slices on stage 2), so no SM gets a whole extra slice.
+// A producer warp loads the slices of the CTA's range into a two-buffer ring
+// (each slice's K and V are one 4-D TMA box each: the whole map of one head,
+// 64-byte token rows in map order, 64-byte swizzle), so the next slice lands
+// while the compute warps work on the current one; the compute warps take
+// the range's items in turn and release a buffer once done with its slice.
+// Every wait is bounded (on expiry: kDevTimeout, all roles stop, copies in
+// flight are waited for).  Routes: a region listed more than once counts
+// once (later listings are masked), and a query region with an out-of-range
+// route is reported (BRA_ERR_BAD_ROUTE) and not written.
 #include <cuda.h>
 #include <stdlib.h>
 
@@ -37,11 +41,14 @@
 namespace bra {
 namespace {
 
-constexpr int kWarps = 12;
-constexpr int kThreads = 32 * kWarps;
+// Compute warps per CTA (one CTA per SM): 23 where a warp's S row block fits
+// in the register share of 24 warps (up to 64 keys per query), 12 for 128.
+// One more warp is the producer.
+constexpr int compute_warps_for(int kn) { return kn <= 64 ? 23 : 12; }
+constexpr uint32_t kMaxSliceBytes = 55u * 1024u;  // K or V of one slice; two slices of K + V resident
+
 constexpr uint32_t kWait = 1u << 22;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kMaxSliceBytes = 2u * 50u * 1024u;  // K + V: two CTAs per SM
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -70,193 +77,267 @@ __device__ __forceinline__ uint32_t swz64(uint32_t base, int row, int c) {
     return base + (uint32_t)row * 64u + (uint32_t)((c ^ ((row >> 1) & 3)) << 4);
 }
 
+struct RingBarriers {
+    uint64_t full[2];   // slice buffer b holds its slice (TMA bytes landed)
+    uint64_t empty[2];  // every compute warp is done with slice buffer b
+    int issued;         // slices whose loads the producer has issued
+    int abort;
+};
+
+__device__ __forceinline__ bool ring_aborted(RingBarriers* rb) {
+    return *reinterpret_cast<volatile int*>(&rb->abort) != 0;
+}
+__device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, RingBarriers* rb, int* status) {
+    for (uint32_t i = 0; i < kWait; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 63u && ring_aborted(rb)) return false;
+    }
+    raise_status(status, kDevTimeout);
+    *reinterpret_cast<volatile int*>(&rb->abort) = 1;
+    return false;
+}
+
 // KN: keys per query region (topk * n), a multiple of 16, at most 128.
 template <int KN>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(32 * (compute_warps_for(KN) + 1), 1)
 bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
                        __nv_bfloat16* __restrict__ o, Geometry g, int* status) {
     constexpr int NT = KN / 8;  // 8-key column tiles of S
+    constexpr int kCompute = compute_warps_for(KN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t region_bytes = (uint32_t)g.n * 64u;
     const uint32_t slice_bytes = (uint32_t)g.R * region_bytes;
-    const uint32_t k_base = ptx::smem_addr(smem), v_base = k_base + slice_bytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * slice_bytes);
+    const uint32_t ring_base = ptx::smem_addr(smem);  // buffer b: K at ring_base + b * 2 * slice_bytes, then V
+    RingBarriers* rb = reinterpret_cast<RingBarriers*>(smem + 4 * slice_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x, b = bh / g.heads, hd = bh - b * g.heads;
+
+    // n = topk * n / topk with topk * n in {32, 64, 128} and 16 | n, so n (and
+    // with it ws and hs) is a power of two: index arithmetic by shifts
+    const int lg_n = __ffs(g.n) - 1, lg_ws = __ffs(g.ws) - 1;
+    const int lg_chunks = lg_n - 4;  // 16-query chunks per region
+    const int per_slice = g.R << lg_chunks;
+    // this CTA's contiguous share of all (slice, region, chunk) items
+    const long long total = (long long)g.B * g.heads * per_slice;
+    const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+    const int s_first = (int)(lo / per_slice);
+    const int n_slices = hi > lo ? (int)((hi - 1) / per_slice) - s_first + 1 : 0;
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(full, 1);
+        ptx::mbar_init(&rb->full[0], 1);
+        ptx::mbar_init(&rb->full[1], 1);
+        ptx::mbar_init(&rb->empty[0], kCompute);
+        ptx::mbar_init(&rb->empty[1], kCompute);
+        rb->abort = 0;
+        rb->issued = 0;
         ptx::mbar_init_fence();
     }
     __syncthreads();
     grid_dependency_wait();
-    if (warp == 0) {
+
+    if (warp == kCompute) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
             ptx::tma_prefetch_desc(&tk);
             ptx::tma_prefetch_desc(&tv);
-            ptx::mbar_arrive_expect_tx(full, 2u * slice_bytes);
         }
-        __syncwarp();
-        for (int j = lane; j < 2 * g.R; j += 32) {
-            const int r = j >> 1, ri = r / g.S, rj = r - ri * g.S;
-            const bool is_v = j & 1;
-            ptx::tma_load_4d((is_v ? v_base : k_base) + (uint32_t)r * region_bytes,
-                             is_v ? (const void*)&tv : (const void*)&tk, hd * 32, rj * g.ws, ri * g.hs, b, full);
+        for (int k = 0; k < n_slices; ++k) {
+            const int buf = k & 1;
+            if (k >= 2 && !ring_wait(&rb->empty[buf], ((k - 2) >> 1) & 1, rb, status)) break;
+            const int bh = s_first + k, b = bh / g.heads, hd = bh - b * g.heads;
+            const uint32_t k_base = ring_base + (uint32_t)buf * 2u * slice_bytes, v_base = k_base + slice_bytes;
+            // the whole map of one head, token-major (row y * W + x of the buffer)
+            if (lane == 0) {
+                ptx::mbar_arrive_expect_tx(&rb->full[buf], 2u * slice_bytes);
+                ptx::tma_load_4d(k_base, &tk, hd * 32, 0, 0, b, &rb->full[buf]);
+                ptx::tma_load_4d(v_base, &tv, hd * 32, 0, 0, b, &rb->full[buf]);
+            }
+            __syncwarp();
+            if (lane == 0) rb->issued = k + 1;
+        }
+    } else {
+        // --------------------------------------------------------- compute warps
+        const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
+        const float sl = kLog2e * rsqrtf(32.f);
+        constexpr uint32_t kOnes = 0x3f803f80u;   // a bf16 pair of ones: the B operand of the row sums
+        long long it = lo + warp;                 // items lo + warp, lo + warp + kCompute, ...
+        for (int k = 0; k < n_slices; ++k) {
+            const int buf = k & 1;
+            const int bh = s_first + k, b = bh / g.heads, hd = bh - b * g.heads;
+            const long long s_end = hi < (long long)(bh + 1) * per_slice ? hi : (long long)(bh + 1) * per_slice;
+            const uint32_t k_base = ring_base + (uint32_t)buf * 2u * slice_bytes, v_base = k_base + slice_bytes;
+            const int32_t* routes = idx + (size_t)bh * g.R * g.topk;
+            bool landed = false, stop = false;
+            for (; it < s_end; it += kCompute) {
+                const int item = (int)(it - (long long)bh * per_slice);
+                const int r = item >> lg_chunks, ch = item & ((1 << lg_chunks) - 1);
+                // routes of region r: lane m < topk holds route m; live: in range and
+                // its first listing; any route out of range skips the region
+                const int my_r = lane < g.topk ? __ldg(routes + r * g.topk + lane) : 0;
+                const uint32_t badm = __ballot_sync(0xffffffffu, lane < g.topk && (my_r < 0 || my_r >= g.R));
+                if (badm) {
+                    if (lane == 0) raise_status(status, kDevBadRoute);
+                    continue;
+                }
+                bool dup = false;
+                for (int dd = 1; dd < g.topk; ++dd) {
+                    const int other = __shfl_up_sync(0xffffffffu, my_r, dd);
+                    if (dd <= lane && other == my_r) dup = true;
+                }
+                const uint32_t live = __ballot_sync(0xffffffffu, lane < g.topk && !dup);
+                const bool all_live = live == (g.topk >= 32 ? 0xffffffffu : (1u << g.topk) - 1u);
+                // buffer row of token (0, 0) of route ``lane``'s region
+                const int my_base = (my_r / g.S) * g.hs * g.W + (my_r - (my_r / g.S) * g.S) * g.ws;
+                // this chunk's 16 query tokens: rows t0 and t0 + 8 of the region
+                const int ri = r / g.S, rj = r - ri * g.S;
+                const int t0 = ch * 16 + gq, t1 = t0 + 8;
+                const size_t corner = ((size_t)b * g.H + (size_t)ri * g.hs) * g.W + (size_t)rj * g.ws;
+                const size_t orow0 = (corner + (size_t)(t0 >> lg_ws) * g.W + (t0 & (g.ws - 1))) * g.C + (size_t)hd * 32;
+                const size_t orow1 = (corner + (size_t)(t1 >> lg_ws) * g.W + (t1 & (g.ws - 1))) * g.C + (size_t)hd * 32;
+                uint32_t qa[2][4];
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc) {
+                    const int c0 = 16 * kc + 2 * tq;
+                    qa[kc][0] = __ldg(reinterpret_cast<const uint32_t*>(q + orow0 + c0));
+                    qa[kc][1] = __ldg(reinterpret_cast<const uint32_t*>(q + orow1 + c0));
+                    qa[kc][2] = __ldg(reinterpret_cast<const uint32_t*>(q + orow0 + c0 + 8));
+                    qa[kc][3] = __ldg(reinterpret_cast<const uint32_t*>(q + orow1 + c0 + 8));
+                }
+                if (!landed) {
+                    if (!ring_wait(&rb->full[buf], (k >> 1) & 1, rb, status)) {
+                        stop = true;
+                        break;
+                    }
+                    landed = true;
+                }
+                // S = Q K^T over the routed keys: column tile j is keys 8j..8j+7 of the
+                // stacked list (route j*8/n, key (8j) % n of that region)
+                float s[NT][4];
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+                    const int m = (8 * j) >> lg_n;  // route of the tile (the same for every lane)
+                    const int base = __shfl_sync(0xffffffffu, my_base, m < 32 ? m : 0);
+                    const int kk = ((8 * j) & (g.n - 1)) + (lane & 7);  // key of the region
+                    const int row = base + (kk >> lg_ws) * g.W + (kk & (g.ws - 1));
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(swz64(k_base, row, lane >> 3), b0, b1, b2, b3);
+                    mma16816(s[j], qa[0][0], qa[0][1], qa[0][2], qa[0][3], b0, b1);
+                    mma16816(s[j], qa[1][0], qa[1][1], qa[1][2], qa[1][3], b2, b3);
+                }
+                // masked base-2 softmax over each row (rows gq and gq + 8; a row's 16
+                // values of a tile sit in the 4 lanes of its group)
+                if (!all_live) {
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) {
+                        const int m = (8 * j) >> lg_n;
+                        if (!((live >> m) & 1u)) s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
+                    }
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+                    mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+                }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float m0 = mx0 * sl, m1 = mx1 * sl;
+                // P as bf16 pairs (the A operand of P V)
+                uint32_t pa[NT][2];
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    pa[j][0] = ptx::pack_bf16x2(ptx::ex2(fmaf(s[j][0], sl, -m0)), ptx::ex2(fmaf(s[j][1], sl, -m0)));
+                    pa[j][1] = ptx::pack_bf16x2(ptx::ex2(fmaf(s[j][2], sl, -m1)), ptx::ex2(fmaf(s[j][3], sl, -m1)));
+                }
+                // O = P V: 16 keys per step (tiles 2k, 2k + 1 of P), V rows of the routed
+                // region read transposed by ldmatrix; 4 tiles of 8 channels.  The row
+                // sums of the bf16 P come from one more product per step against ones
+                // (every column of ls holds its row's sum).
+                float acc[4][4], ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) acc[nn][0] = acc[nn][1] = acc[nn][2] = acc[nn][3] = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < NT / 2; ++kk) {
+                    const int m = (16 * kk) >> lg_n;
+                    const int base = __shfl_sync(0xffffffffu, my_base, m < 32 ? m : 0);
+                    mma16816(ls, pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], kOnes, kOnes);
+                    // matrices: (keys 0-7, ch c..c+7), (keys 8-15, ch c..), (keys 0-7, ch c+8..), (keys 8-15, ch c+8..)
+                    const int key = ((16 * kk) & (g.n - 1)) + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int row = base + (key >> lg_ws) * g.W + (key & (g.ws - 1));
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(swz64(v_base, row, 2 * half + (lane >> 4)), b0, b1, b2, b3);
+                        mma16816(acc[2 * half], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
+                        mma16816(acc[2 * half + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1],
+                                 b2, b3);
+                    }
+                }
+                // O rows gq and gq + 8: channels 8n + 2tq, 8n + 2tq + 1
+                const float i0 = ls[0] > 0.f ? 1.f / ls[0] : 0.f, i1 = ls[2] > 0.f ? 1.f / ls[2] : 0.f;
+                if (!in_bounds((orow0 > orow1 ? orow0 : orow1) + 31, map_elems(g), status)) continue;
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) {
+                    const int c = 8 * nn + 2 * tq;
+                    __stcs(reinterpret_cast<uint32_t*>(o + orow0 + c), ptx::pack_bf16x2(acc[nn][0] * i0, acc[nn][1] * i0));
+                    __stcs(reinterpret_cast<uint32_t*>(o + orow1 + c), ptx::pack_bf16x2(acc[nn][2] * i1, acc[nn][3] * i1));
+                }
+            }
+            if (stop) break;
+            // a warp with no item in this slice still waits for its load before
+            // releasing the buffer: an early release would count toward this
+            // buffer's previous slice
+            if (!landed && !ring_wait(&rb->full[buf], (k >> 1) & 1, rb, status)) break;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&rb->empty[buf]);
         }
     }
-
-    const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
-    const float sl = kLog2e * rsqrtf(32.f);
-    const int chunks = g.n / 16;              // 16-query chunks per region
-    const int items = g.R * chunks;
-    const int32_t* routes = idx + (size_t)bh * g.R * g.topk;
-    bool landed = false;
-    for (int it = warp; it < items; it += kWarps) {
-        const int r = it / chunks, ch = it - r * chunks;
-        // routes of region r: lane m < topk holds route m; live: in range and
-        // its first listing; any route out of range skips the region
-        const int my_r = lane < g.topk ? __ldg(routes + r * g.topk + lane) : 0;
-        const uint32_t badm = __ballot_sync(0xffffffffu, lane < g.topk && (my_r < 0 || my_r >= g.R));
-        if (badm) {
-            if (lane == 0) raise_status(status, kDevBadRoute);
-            continue;
-        }
-        bool dup = false;
-        for (int dd = 1; dd < g.topk; ++dd) {
-            const int other = __shfl_up_sync(0xffffffffu, my_r, dd);
-            if (dd <= lane && other == my_r) dup = true;
-        }
-        const uint32_t live = __ballot_sync(0xffffffffu, lane < g.topk && !dup);
-        const int my_base = my_r * g.n;  // first slice row of route ``lane``
-        // this chunk's 16 query tokens: rows t0 + gq and t0 + gq + 8 of the region
-        const int t0 = ch * 16;
-        const size_t orow0 = token_offset(g, b, r, t0 + gq) + (size_t)hd * 32;
-        const size_t orow1 = token_offset(g, b, r, t0 + gq + 8) + (size_t)hd * 32;
-        uint32_t qa[2][4];
-#pragma unroll
-        for (int kc = 0; kc < 2; ++kc) {
-            const int c0 = 16 * kc + 2 * tq;
-            qa[kc][0] = __ldg(reinterpret_cast<const uint32_t*>(q + orow0 + c0));
-            qa[kc][1] = __ldg(reinterpret_cast<const uint32_t*>(q + orow1 + c0));
-            qa[kc][2] = __ldg(reinterpret_cast<const uint32_t*>(q + orow0 + c0 + 8));
-            qa[kc][3] = __ldg(reinterpret_cast<const uint32_t*>(q + orow1 + c0 + 8));
-        }
-        if (!landed) {
-            if (!ptx::mbar_wait(full, 0, kWait)) {
-                if (lane == 0) raise_status(status, kDevTimeout);
-                break;
-            }
-            landed = true;
-        }
-        // S = Q K^T over the routed keys: column tile j is keys 8j..8j+7 of the
-        // stacked list (route j*8/n, key (8j) % n of that region)
-        float s[NT][4];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-            const int m = (8 * j) / g.n;  // route of the tile (the same for every lane)
-            const int base = __shfl_sync(0xffffffffu, my_base, m < 32 ? m : 0);
-            if (8 * j >= g.topk * g.n) continue;
-            const int row = base + (8 * j) % g.n + (lane & 7);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(swz64(k_base, row, lane >> 3), b0, b1, b2, b3);
-            mma16816(s[j], qa[0][0], qa[0][1], qa[0][2], qa[0][3], b0, b1);
-            mma16816(s[j], qa[1][0], qa[1][1], qa[1][2], qa[1][3], b2, b3);
-        }
-        // masked base-2 softmax over each row (rows gq and gq + 8; a row's 16
-        // values of a tile sit in the 4 lanes of its group)
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            const int m = (8 * j) / g.n;
-            const bool on = 8 * j < g.topk * g.n && ((live >> m) & 1u);
-            if (!on) s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
-            mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
-            mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float m0 = mx0 * sl, m1 = mx1 * sl;
-        // P as bf16 pairs (the A operand of P V), and the row sums of those bf16 values
-        uint32_t pa[NT][2];
-        float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            pa[j][0] = ptx::pack_bf16x2(ptx::ex2(fmaf(s[j][0], sl, -m0)), ptx::ex2(fmaf(s[j][1], sl, -m0)));
-            pa[j][1] = ptx::pack_bf16x2(ptx::ex2(fmaf(s[j][2], sl, -m1)), ptx::ex2(fmaf(s[j][3], sl, -m1)));
-            l0 += __uint_as_float(pa[j][0] << 16) + __uint_as_float(pa[j][0] & 0xffff0000u);
-            l1 += __uint_as_float(pa[j][1] << 16) + __uint_as_float(pa[j][1] & 0xffff0000u);
-        }
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-        // O = P V: 16 keys per step (tiles 2k, 2k + 1 of P), V rows of the routed
-        // region read transposed by ldmatrix; 4 tiles of 8 channels
-        float acc[4][4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < NT / 2; ++kk) {
-            const int m = (16 * kk) / g.n;
-            const int base = __shfl_sync(0xffffffffu, my_base, m < 32 ? m : 0);
-            if (16 * kk >= g.topk * g.n) continue;
-            // matrices: (keys 0-7, ch c..c+7), (keys 8-15, ch c..), (keys 0-7, ch c+8..), (keys 8-15, ch c+8..)
-            const int row = base + (16 * kk) % g.n + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(swz64(v_base, row, 2 * half + (lane >> 4)), b0, b1, b2, b3);
-                mma16816(acc[2 * half], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
-                mma16816(acc[2 * half + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2,
-                         b3);
-            }
-        }
-        // O rows gq and gq + 8: channels 8n + 2tq, 8n + 2tq + 1
-        const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-        if (!in_bounds((orow0 > orow1 ? orow0 : orow1) + 31, map_elems(g), status)) continue;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            const int c = 8 * n + 2 * tq;
-            __stcs(reinterpret_cast<uint32_t*>(o + orow0 + c), ptx::pack_bf16x2(acc[n][0] * i0, acc[n][1] * i0));
-            __stcs(reinterpret_cast<uint32_t*>(o + orow1 + c), ptx::pack_bf16x2(acc[n][2] * i1, acc[n][3] * i1));
-        }
-    }
-    // every copy this CTA issued must land before it exits
-    if (!landed && warp == 0 && lane == 0) ptx::mbar_wait(full, 0, kWait);
     __syncthreads();
+    // every copy this CTA issued must land before it exits: the last use of each
+    // buffer is its latest phase (already complete unless a wait gave up)
+    if (threadIdx.x == 0) {
+        const int issued = rb->issued;
+        for (int k = issued - 2 < 0 ? 0 : issued - 2; k < issued; ++k)
+            ptx::mbar_wait(&rb->full[k & 1], (k >> 1) & 1, kWait);
+    }
 }
 
 }  // namespace
 
 bool attend_warp_covers(const Geometry& g) {
     const int kn = g.topk * g.n;
-    return g.d == 32 && g.n % 16 == 0 && kn <= 128 && (kn == 32 || kn == 64 || kn == 128) &&
-           2u * (uint32_t)g.R * (uint32_t)g.n * 64u <= kMaxSliceBytes;
+    // kn in {32, 64, 128} and 16 | n make n, ws and hs powers of two (checked
+    // anyway: the kernel's index arithmetic relies on it)
+    return g.d == 32 && g.n % 16 == 0 && (kn == 32 || kn == 64 || kn == 128) && (g.n & (g.n - 1)) == 0 &&
+           (g.ws & (g.ws - 1)) == 0 && g.W <= 256 && g.H <= 256 &&  // one TMA box per map
+           (uint32_t)g.R * (uint32_t)g.n * 64u <= kMaxSliceBytes;
 }
 
 bra_status attend_warp_launch(const Geometry& g, const void* q, const void* k, const void* v, const int32_t* idx,
                               void* o, int* status, cudaStream_t stream) {
     if (!attend_warp_covers(g)) return BRA_ERR_UNSUPPORTED;
     CUtensorMap tk, tv;
-    if (!encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs, 32) ||
-        !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.ws, g.hs, 32))
+    if (!encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.W, g.H, 32) ||
+        !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.W, g.H, 32))
         return BRA_ERR_UNSUPPORTED;
-    const long long slices = (long long)g.B * g.heads;
-    if (slices > 0x7fffffffLL) return BRA_ERR_UNSUPPORTED;
-    const uint32_t smem = 2u * (uint32_t)g.R * (uint32_t)g.n * 64u + 64u + 1024u;
+    const long long items = (long long)g.B * g.heads * g.R * (g.n / 16);
+    const int sms = sm_count();
+    if (sms <= 0) return BRA_ERR_CUDA;
+    const int grid = items < sms ? (int)items : sms;
+    const uint32_t smem = 4u * (uint32_t)g.R * (uint32_t)g.n * 64u + (uint32_t)sizeof(RingBarriers) + 1024u;
     using KernelFn = void (*)(CUtensorMap, CUtensorMap, const __nv_bfloat16*, const int32_t*, __nv_bfloat16*, Geometry,
                               int*);
     const int kn = g.topk * g.n;
+    const unsigned threads = 32u * (unsigned)(compute_warps_for(kn) + 1);
     const KernelFn kernel = kn == 32 ? bra_attend_warp_kernel<32>
                                      : (kn == 64 ? bra_attend_warp_kernel<64> : bra_attend_warp_kernel<128>);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return BRA_ERR_CUDA;
-    const cudaError_t e = launch_after_previous(kernel, dim3((unsigned)slices), dim3(kThreads), smem, stream, tk, tv,
+    const cudaError_t e = launch_after_previous(kernel, dim3((unsigned)grid), dim3(threads), smem, stream, tk, tv,
                                                 static_cast<const __nv_bfloat16*>(q), idx,
                                                 static_cast<__nv_bfloat16*>(o), g, status);
     return e == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
