@@ -68,8 +68,6 @@ struct Barriers {
     uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full[kGroups][2], s_free[kGroups][2], p_full[kGroups][2], o_full[kGroups][2];
     uint64_t drain[2];
-    uint32_t live[kGroups];               // bit m: route m in range and its first listing
-    int bad[kGroups];                     // some route of the tile is out of range
     uint32_t tmem;
     int abort;
 };
@@ -114,6 +112,25 @@ __device__ __forceinline__ void tile_coords(const FlashPlan& p, const Geometry& 
     const int rr = t / p.parts;
     r = rr % g.R;
     bh = rr / g.R;
+}
+
+// The tile's routes as the softmax sees them: bit m of ``live`` set when
+// route m is in range and its first listing; ``bad`` when any route is out
+// of range.  Every lane of the calling warp gets the same result.  (Each
+// softmax warp reads them itself: a value handed over by the producer could
+// be overwritten for the group's next tile before a short tile's softmax has
+// read it.)
+__device__ __forceinline__ void tile_routes(const Geometry& g, const int32_t* __restrict__ idx, int bh, int r,
+                                            int lane, uint32_t& live, bool& bad) {
+    int my_r = lane < g.topk ? __ldg(idx + ((size_t)bh * g.R + r) * g.topk + lane) : 0;
+    const bool out = lane < g.topk && (my_r < 0 || my_r >= g.R);
+    bad = __ballot_sync(0xffffffffu, out) != 0u;
+    bool dup = false;
+    for (int dd = 1; dd < g.topk; ++dd) {
+        const int other = __shfl_up_sync(0xffffffffu, my_r, dd);
+        if (dd <= lane && other == my_r) dup = true;
+    }
+    live = __ballot_sync(0xffffffffu, lane < g.topk && !out && !dup);
 }
 
 // Columns c0 .. c0 + 63 of this warp's TMEM rows at ``taddr``: four x16 loads,
@@ -196,27 +213,12 @@ bra_attend_flash_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             tile_coords(p, g, st.tile, bh, r, part);
             const int b = bh / g.heads, hd = bh - b * g.heads;
             if (st.b == 0) {
-                // routes of the tile (lane m < topk holds route m), the live mask
-                // and the bad flag for the softmax group; then the tile's Q box
+                // routes of the tile (lane m < topk holds route m), then its Q box
                 if (use > 0 && !wait_or_abort(&sb->q_empty[grp], (use - 1) & 1, sb, status)) break;
                 int my_r = lane < g.topk ? __ldg(idx + ((size_t)bh * g.R + r) * g.topk + lane) : 0;
-                const bool bad = lane < g.topk && (my_r < 0 || my_r >= g.R);
-                const uint32_t badm = __ballot_sync(0xffffffffu, bad);
-                if (bad) my_r = 0;
-                bool dup = false;
-                for (int dd = 1; dd < g.topk; ++dd) {
-                    const int other = __shfl_up_sync(0xffffffffu, my_r, dd);
-                    if (dd <= lane && other == my_r) dup = true;
-                }
-                const uint32_t live = __ballot_sync(0xffffffffu, lane < g.topk && !bad && !dup);
+                if (my_r < 0 || my_r >= g.R) my_r = 0;  // the softmax reports and discards the tile
                 if (grp) my_r1 = my_r;
                 else my_r0 = my_r;
-                if (lane == 0) {
-                    sb->live[grp] = live;
-                    sb->bad[grp] = badm != 0u;
-                    if (badm) raise_status(status, kDevBadRoute);
-                }
-                __syncwarp();
                 if (lane == 0) {
                     ptx::mbar_arrive_expect_tx(&sb->q_full[grp], kQBytes);
                     const int ri = r / g.S, rj = r - ri * g.S;
@@ -312,8 +314,12 @@ bra_attend_flash_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
 #pragma unroll
             for (int c = 0; c < 32; ++c) acc[c] = 0.f;
             float alpha_prev = 0.f;  // rescale of the block whose O is folded next
-            uint32_t live = 0u;      // the tile's live routes and bad flag, read at its first block:
-            bool bad = false;        // the producer rewrites them for the group's next tile
+            int tbh = 0, tr = 0, tpart = 0;
+            tile_coords(p, g, tile, tbh, tr, tpart);
+            uint32_t live = 0u;
+            bool bad = false;
+            tile_routes(g, idx, tbh, tr, lane, live, bad);
+            if (bad && qd == 0 && lane == 0) raise_status(status, kDevBadRoute);
             // fold O_blk of the group's k-th block into acc (after its P V is done)
             auto fold = [&](int k, float alpha) -> bool {
                 const int buf = k & 1;
@@ -342,10 +348,6 @@ bra_attend_flash_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                     break;
                 }
                 ptx::tc_fence_after();
-                if (b == 0) {
-                    live = *reinterpret_cast<volatile uint32_t*>(&sb->live[grp]);
-                    bad = *reinterpret_cast<volatile int*>(&sb->bad[grp]) != 0;
-                }
                 const bool on = (live >> (b / p.kb)) & 1u;  // a repeated listing contributes nothing
                 const uint32_t sa = tmem + lane_addr + (uint32_t)(grp * 2 + buf) * 128u;
                 float mb = -INFINITY;
@@ -403,11 +405,9 @@ bra_attend_flash_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             if (!ok) break;
             // the tile's last block, then O = acc / l
             if (!fold(use * p.nb + p.nb - 1, alpha_prev)) break;
-            int bh = 0, r = 0, part = 0;
-            tile_coords(p, g, tile, bh, r, part);
-            const int b = bh / g.heads, hd = bh - b * g.heads;
+            const int b = tbh / g.heads, hd = tbh - b * g.heads;
             const bool write = !bad && l_acc > 0.f;
-            const size_t ooff = token_offset(g, b, r, part * 128 + row) + (size_t)hd * 32;
+            const size_t ooff = token_offset(g, b, tr, tpart * 128 + row) + (size_t)hd * 32;
             if (write && in_bounds(ooff + 31, map_elems(g), status)) {
                 const float inv = 1.f / l_acc;
                 int4* dst = reinterpret_cast<int4*>(o + ooff);

@@ -21,11 +21,16 @@
 // Work: persistent, one CTA per SM.  All (slice, region, 16-query chunk)
 // items are split into equal contiguous ranges, one per CTA (a CTA's range
 // spans two or three slices on stage 2), so no SM gets a whole extra slice.
-// A producer warp loads the slices of the CTA's range into a two-buffer ring
-// (each slice's K and V are one 4-D TMA box each: the whole map of one head,
-// 64-byte token rows in map order, 64-byte swizzle), so the next slice lands
-// while the compute warps work on the current one; the compute warps take
-// the range's items in turn and release a buffer once done with its slice.
+// A producer warp loads the slices of the CTA's range into a two-buffer ring,
+// so the next slice lands while the compute warps work on the current one;
+// the compute warps take the range's items in turn and release a buffer once
+// done with its slice.  A slice's K (and its V) is one 5-D TMA box: the map
+// viewed as (channel, x in region, y in region, region column, image x region
+// row) lands region-major, region r's n tokens in 64-byte rows r * n .. r * n
+// + n - 1 (64-byte swizzle).  Routed regions then start at multiples of 16
+// rows, so each lane's ldmatrix addresses are its route's base plus constants
+// (the swizzle included) and the per-tile offsets are compile-time constants
+// of the region size.
 // Every wait is bounded (on expiry: kDevTimeout, all roles stop, copies in
 // flight are waited for).  Routes: a region listed more than once counts
 // once (later listings are masked), and a query region with an out-of-range
@@ -41,10 +46,10 @@
 namespace bra {
 namespace {
 
-// Compute warps per CTA (one CTA per SM): 23 where a warp's S row block fits
-// in the register share of 24 warps (up to 64 keys per query), 12 for 128.
-// One more warp is the producer.
-constexpr int compute_warps_for(int kn) { return kn <= 64 ? 23 : 12; }
+// Compute warps per CTA (one CTA per SM), one more warp being the producer:
+// 19 for up to 64 keys per query, 12 for 128 (a warp's S row block needs
+// more registers).
+constexpr int compute_warps_for(int kn) { return kn <= 64 ? 19 : 12; }
 constexpr uint32_t kMaxSliceBytes = 55u * 1024u;  // K or V of one slice; two slices of K + V resident
 
 constexpr uint32_t kWait = 1u << 22;
@@ -97,33 +102,44 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, RingBa
     return false;
 }
 
-// KN: keys per query region (topk * n), a multiple of 16, at most 128.
-template <int KN>
-__global__ void __launch_bounds__(32 * (compute_warps_for(KN) + 1), 1)
+// KN: keys per query region (topk * n); N: tokens per region (a power of two,
+// 16..KN).  Both are template parameters so that the route and in-region
+// offset of every 8-key tile of S and every 16-key step of P V are constants.
+// Registers per thread: the most that lets one CTA of compute_warps_for(KN) + 1
+// warps fit (warps are spread over the SM's four 16 K-register files: 20
+// warps put 5 on each, 5 x 32 x 96 <= 16 K; 13 warps put 4 on one, 4 x 32 x 128).
+constexpr int max_regs_for(int kn) { return kn <= 64 ? 96 : 128; }
+
+template <int KN, int N>
+__global__ void __maxnreg__(max_regs_for(KN))
 bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ idx,
                        __nv_bfloat16* __restrict__ o, Geometry g, int* status) {
-    constexpr int NT = KN / 8;  // 8-key column tiles of S
+    constexpr int NT = KN / 8;     // 8-key column tiles of S
+    constexpr int TOPK = KN / N;   // routes per query region
+    constexpr int CHUNKS = N / 16; // 16-query chunks per region
     constexpr int kCompute = compute_warps_for(KN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t region_bytes = (uint32_t)g.n * 64u;
-    const uint32_t slice_bytes = (uint32_t)g.R * region_bytes;
+    const uint32_t slice_bytes = (uint32_t)g.R * (uint32_t)N * 64u;
     const uint32_t ring_base = ptx::smem_addr(smem);  // buffer b: K at ring_base + b * 2 * slice_bytes, then V
     RingBarriers* rb = reinterpret_cast<RingBarriers*>(smem + 4 * slice_bytes);
+    int* qcorner = reinterpret_cast<int*>(smem + 4 * slice_bytes + ((sizeof(RingBarriers) + 15) & ~size_t(15)));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // n = topk * n / topk with topk * n in {32, 64, 128} and 16 | n, so n (and
-    // with it ws and hs) is a power of two: index arithmetic by shifts
-    const int lg_n = __ffs(g.n) - 1, lg_ws = __ffs(g.ws) - 1;
-    const int lg_chunks = lg_n - 4;  // 16-query chunks per region
-    const int per_slice = g.R << lg_chunks;
-    // this CTA's contiguous share of all (slice, region, chunk) items
+    const int lg_ws = __ffs(g.ws) - 1;
+    const int per_slice = g.R * CHUNKS;
+    // this CTA's contiguous share of all (slice, region, chunk) items (the
+    // host checks that their number fits an int)
     const long long total = (long long)g.B * g.heads * per_slice;
-    const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
-    const int s_first = (int)(lo / per_slice);
-    const int n_slices = hi > lo ? (int)((hi - 1) / per_slice) - s_first + 1 : 0;
+    const int lo = (int)(total * blockIdx.x / gridDim.x), hi = (int)(total * (blockIdx.x + 1) / gridDim.x);
+    const int s_first = lo / per_slice;
+    const int n_slices = hi > lo ? (hi - 1) / per_slice - s_first + 1 : 0;
 
+    // map offset of each query region's token (0, 0)
+    for (int r = threadIdx.x; r < g.R; r += blockDim.x) {
+        const int ri = r / g.S;
+        qcorner[r] = ri * g.hs * g.W + (r - ri * g.S) * g.ws;
+    }
     if (threadIdx.x == 0) {
         ptx::mbar_init(&rb->full[0], 1);
         ptx::mbar_init(&rb->full[1], 1);
@@ -147,54 +163,64 @@ bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_cons
             if (k >= 2 && !ring_wait(&rb->empty[buf], ((k - 2) >> 1) & 1, rb, status)) break;
             const int bh = s_first + k, b = bh / g.heads, hd = bh - b * g.heads;
             const uint32_t k_base = ring_base + (uint32_t)buf * 2u * slice_bytes, v_base = k_base + slice_bytes;
-            // the whole map of one head, token-major (row y * W + x of the buffer)
+            // one head of every region of the image, region-major: region r's
+            // tokens are buffer rows r * N .. r * N + N - 1 in their in-region order
             if (lane == 0) {
                 ptx::mbar_arrive_expect_tx(&rb->full[buf], 2u * slice_bytes);
-                ptx::tma_load_4d(k_base, &tk, hd * 32, 0, 0, b, &rb->full[buf]);
-                ptx::tma_load_4d(v_base, &tv, hd * 32, 0, 0, b, &rb->full[buf]);
+                ptx::tma_load_5d(k_base, &tk, hd * 32, 0, 0, 0, b * g.S, &rb->full[buf]);
+                ptx::tma_load_5d(v_base, &tv, hd * 32, 0, 0, 0, b * g.S, &rb->full[buf]);
+                rb->issued = k + 1;
             }
             __syncwarp();
-            if (lane == 0) rb->issued = k + 1;
         }
     } else {
         // --------------------------------------------------------- compute warps
         const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
         const float sl = kLog2e * rsqrtf(32.f);
         constexpr uint32_t kOnes = 0x3f803f80u;   // a bf16 pair of ones: the B operand of the row sums
-        long long it = lo + warp;                 // items lo + warp, lo + warp + kCompute, ...
+        // Shared-memory byte offsets of this lane's ldmatrix rows.  A routed
+        // region starts at a multiple of 16 rows and every tile or step at a
+        // multiple of 8 rows inside it, so the 64-byte swizzle (chunk XOR bits
+        // 1-2 of the row) depends on the lane alone.
+        const int kl = lane & 7, vrow = kl + ((lane >> 3) & 1) * 8;
+        const uint32_t s_lane = (uint32_t)kl * 64u + ((uint32_t)((lane >> 3) ^ ((kl >> 1) & 3)) << 4);
+        const uint32_t v_lane0 = (uint32_t)vrow * 64u + ((uint32_t)((0 + (lane >> 4)) ^ ((kl >> 1) & 3)) << 4);
+        const uint32_t v_lane1 = (uint32_t)vrow * 64u + ((uint32_t)((2 + (lane >> 4)) ^ ((kl >> 1) & 3)) << 4);
+        int it = lo + warp;  // items lo + warp, lo + warp + kCompute, ...
         for (int k = 0; k < n_slices; ++k) {
             const int buf = k & 1;
             const int bh = s_first + k, b = bh / g.heads, hd = bh - b * g.heads;
-            const long long s_end = hi < (long long)(bh + 1) * per_slice ? hi : (long long)(bh + 1) * per_slice;
-            const uint32_t k_base = ring_base + (uint32_t)buf * 2u * slice_bytes, v_base = k_base + slice_bytes;
-            const int32_t* routes = idx + (size_t)bh * g.R * g.topk;
+            const int s_end = hi < (bh + 1) * per_slice ? hi : (bh + 1) * per_slice;
+            const uint32_t k_base = ring_base + (uint32_t)buf * 2u * slice_bytes;
+            const int32_t* routes = idx + (size_t)bh * g.R * TOPK;
+            const size_t img = (size_t)b * g.H * g.W;
             bool landed = false, stop = false;
             for (; it < s_end; it += kCompute) {
-                const int item = (int)(it - (long long)bh * per_slice);
-                const int r = item >> lg_chunks, ch = item & ((1 << lg_chunks) - 1);
+                const int item = it - bh * per_slice;
+                const int r = item / CHUNKS, ch = item - r * CHUNKS;
                 // routes of region r: lane m < topk holds route m; live: in range and
                 // its first listing; any route out of range skips the region
-                const int my_r = lane < g.topk ? __ldg(routes + r * g.topk + lane) : 0;
-                const uint32_t badm = __ballot_sync(0xffffffffu, lane < g.topk && (my_r < 0 || my_r >= g.R));
+                const int my_r = lane < TOPK ? __ldg(routes + r * TOPK + lane) : 0;
+                const uint32_t badm = __ballot_sync(0xffffffffu, lane < TOPK && (my_r < 0 || my_r >= g.R));
                 if (badm) {
                     if (lane == 0) raise_status(status, kDevBadRoute);
                     continue;
                 }
                 bool dup = false;
-                for (int dd = 1; dd < g.topk; ++dd) {
+#pragma unroll
+                for (int dd = 1; dd < TOPK; ++dd) {
                     const int other = __shfl_up_sync(0xffffffffu, my_r, dd);
                     if (dd <= lane && other == my_r) dup = true;
                 }
-                const uint32_t live = __ballot_sync(0xffffffffu, lane < g.topk && !dup);
-                const bool all_live = live == (g.topk >= 32 ? 0xffffffffu : (1u << g.topk) - 1u);
-                // buffer row of token (0, 0) of route ``lane``'s region
-                const int my_base = (my_r / g.S) * g.hs * g.W + (my_r - (my_r / g.S) * g.S) * g.ws;
+                const uint32_t live = __ballot_sync(0xffffffffu, lane < TOPK && !dup);
+                constexpr uint32_t kAll = TOPK >= 32 ? 0xffffffffu : (1u << TOPK) - 1u;
+                // K of route ``lane`` starts at this byte (V one slice further)
+                const uint32_t my_kb = k_base + (uint32_t)my_r * (uint32_t)N * 64u;
                 // this chunk's 16 query tokens: rows t0 and t0 + 8 of the region
-                const int ri = r / g.S, rj = r - ri * g.S;
                 const int t0 = ch * 16 + gq, t1 = t0 + 8;
-                const size_t corner = ((size_t)b * g.H + (size_t)ri * g.hs) * g.W + (size_t)rj * g.ws;
-                const size_t orow0 = (corner + (size_t)(t0 >> lg_ws) * g.W + (t0 & (g.ws - 1))) * g.C + (size_t)hd * 32;
-                const size_t orow1 = (corner + (size_t)(t1 >> lg_ws) * g.W + (t1 & (g.ws - 1))) * g.C + (size_t)hd * 32;
+                const size_t corner = img + (size_t)qcorner[r];
+                const size_t orow0 = (corner + (size_t)((t0 >> lg_ws) * g.W + (t0 & (g.ws - 1)))) * g.C + (size_t)hd * 32;
+                const size_t orow1 = (corner + (size_t)((t1 >> lg_ws) * g.W + (t1 & (g.ws - 1)))) * g.C + (size_t)hd * 32;
                 uint32_t qa[2][4];
 #pragma unroll
                 for (int kc = 0; kc < 2; ++kc) {
@@ -204,6 +230,9 @@ bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_cons
                     qa[kc][2] = __ldg(reinterpret_cast<const uint32_t*>(q + orow0 + c0 + 8));
                     qa[kc][3] = __ldg(reinterpret_cast<const uint32_t*>(q + orow1 + c0 + 8));
                 }
+                uint32_t kb[TOPK];
+#pragma unroll
+                for (int m = 0; m < TOPK; ++m) kb[m] = __shfl_sync(0xffffffffu, my_kb, m);
                 if (!landed) {
                     if (!ring_wait(&rb->full[buf], (k >> 1) & 1, rb, status)) {
                         stop = true;
@@ -212,28 +241,22 @@ bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_cons
                     landed = true;
                 }
                 // S = Q K^T over the routed keys: column tile j is keys 8j..8j+7 of the
-                // stacked list (route j*8/n, key (8j) % n of that region)
+                // stacked list (route 8j / N, keys (8j) % N .. of that region)
                 float s[NT][4];
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-                    const int m = (8 * j) >> lg_n;  // route of the tile (the same for every lane)
-                    const int base = __shfl_sync(0xffffffffu, my_base, m < 32 ? m : 0);
-                    const int kk = ((8 * j) & (g.n - 1)) + (lane & 7);  // key of the region
-                    const int row = base + (kk >> lg_ws) * g.W + (kk & (g.ws - 1));
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4(swz64(k_base, row, lane >> 3), b0, b1, b2, b3);
+                    ldsm_x4(kb[(8 * j) / N] + (uint32_t)((8 * j) % N) * 64u + s_lane, b0, b1, b2, b3);
                     mma16816(s[j], qa[0][0], qa[0][1], qa[0][2], qa[0][3], b0, b1);
                     mma16816(s[j], qa[1][0], qa[1][1], qa[1][2], qa[1][3], b2, b3);
                 }
                 // masked base-2 softmax over each row (rows gq and gq + 8; a row's 16
                 // values of a tile sit in the 4 lanes of its group)
-                if (!all_live) {
+                if (live != kAll) {
 #pragma unroll
-                    for (int j = 0; j < NT; ++j) {
-                        const int m = (8 * j) >> lg_n;
-                        if (!((live >> m) & 1u)) s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
-                    }
+                    for (int j = 0; j < NT; ++j)
+                        if (!((live >> ((8 * j) / N)) & 1u)) s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
                 }
                 float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -253,29 +276,25 @@ bra_attend_warp_kernel(const __grid_constant__ CUtensorMap tk, const __grid_cons
                     pa[j][0] = ptx::pack_bf16x2(ptx::ex2(fmaf(s[j][0], sl, -m0)), ptx::ex2(fmaf(s[j][1], sl, -m0)));
                     pa[j][1] = ptx::pack_bf16x2(ptx::ex2(fmaf(s[j][2], sl, -m1)), ptx::ex2(fmaf(s[j][3], sl, -m1)));
                 }
-                // O = P V: 16 keys per step (tiles 2k, 2k + 1 of P), V rows of the routed
-                // region read transposed by ldmatrix; 4 tiles of 8 channels.  The row
-                // sums of the bf16 P come from one more product per step against ones
-                // (every column of ls holds its row's sum).
+                // O = P V: 16 keys per step (tiles 2kk, 2kk + 1 of P), V rows of the
+                // routed region read transposed by ldmatrix; 4 tiles of 8 channels.
+                // The row sums of the bf16 P come from one more product per step
+                // against ones (every column of ls holds its row's sum).
                 float acc[4][4], ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int nn = 0; nn < 4; ++nn) acc[nn][0] = acc[nn][1] = acc[nn][2] = acc[nn][3] = 0.f;
 #pragma unroll
                 for (int kk = 0; kk < NT / 2; ++kk) {
-                    const int m = (16 * kk) >> lg_n;
-                    const int base = __shfl_sync(0xffffffffu, my_base, m < 32 ? m : 0);
                     mma16816(ls, pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], kOnes, kOnes);
                     // matrices: (keys 0-7, ch c..c+7), (keys 8-15, ch c..), (keys 0-7, ch c+8..), (keys 8-15, ch c+8..)
-                    const int key = ((16 * kk) & (g.n - 1)) + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const int row = base + (key >> lg_ws) * g.W + (key & (g.ws - 1));
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_t(swz64(v_base, row, 2 * half + (lane >> 4)), b0, b1, b2, b3);
-                        mma16816(acc[2 * half], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
-                        mma16816(acc[2 * half + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1],
-                                 b2, b3);
-                    }
+                    const uint32_t vstep = kb[(16 * kk) / N] + slice_bytes + (uint32_t)((16 * kk) % N) * 64u;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vstep + v_lane0, b0, b1, b2, b3);
+                    mma16816(acc[0], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
+                    mma16816(acc[1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
+                    ldsm_x4_t(vstep + v_lane1, b0, b1, b2, b3);
+                    mma16816(acc[2], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
+                    mma16816(acc[3], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
                 }
                 // O rows gq and gq + 8: channels 8n + 2tq, 8n + 2tq + 1
                 const float i0 = ls[0] > 0.f ? 1.f / ls[0] : 0.f, i1 = ls[2] > 0.f ? 1.f / ls[2] : 0.f;
@@ -321,20 +340,33 @@ bra_status attend_warp_launch(const Geometry& g, const void* q, const void* k, c
                               void* o, int* status, cudaStream_t stream) {
     if (!attend_warp_covers(g)) return BRA_ERR_UNSUPPORTED;
     CUtensorMap tk, tv;
-    if (!encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.W, g.H, 32) ||
-        !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.W, g.H, 32))
+    if (!encode_region_major_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs, g.S) ||
+        !encode_region_major_map(&tv, v, g.B, g.H, g.W, g.C, g.ws, g.hs, g.S))
         return BRA_ERR_UNSUPPORTED;
     const long long items = (long long)g.B * g.heads * g.R * (g.n / 16);
+    if (items > 0x7fffffffLL) return BRA_ERR_UNSUPPORTED;
     const int sms = sm_count();
     if (sms <= 0) return BRA_ERR_CUDA;
     const int grid = items < sms ? (int)items : sms;
-    const uint32_t smem = 4u * (uint32_t)g.R * (uint32_t)g.n * 64u + (uint32_t)sizeof(RingBarriers) + 1024u;
+    const uint32_t smem = 4u * (uint32_t)g.R * (uint32_t)g.n * 64u + (((uint32_t)sizeof(RingBarriers) + 15u) & ~15u) +
+                          (uint32_t)g.R * 4u + 1024u;
     using KernelFn = void (*)(CUtensorMap, CUtensorMap, const __nv_bfloat16*, const int32_t*, __nv_bfloat16*, Geometry,
                               int*);
     const int kn = g.topk * g.n;
     const unsigned threads = 32u * (unsigned)(compute_warps_for(kn) + 1);
-    const KernelFn kernel = kn == 32 ? bra_attend_warp_kernel<32>
-                                     : (kn == 64 ? bra_attend_warp_kernel<64> : bra_attend_warp_kernel<128>);
+    KernelFn kernel = nullptr;
+    switch (kn * 1000 + g.n) {
+        case 32016: kernel = bra_attend_warp_kernel<32, 16>; break;
+        case 32032: kernel = bra_attend_warp_kernel<32, 32>; break;
+        case 64016: kernel = bra_attend_warp_kernel<64, 16>; break;
+        case 64032: kernel = bra_attend_warp_kernel<64, 32>; break;
+        case 64064: kernel = bra_attend_warp_kernel<64, 64>; break;
+        case 128016: kernel = bra_attend_warp_kernel<128, 16>; break;
+        case 128032: kernel = bra_attend_warp_kernel<128, 32>; break;
+        case 128064: kernel = bra_attend_warp_kernel<128, 64>; break;
+        case 128128: kernel = bra_attend_warp_kernel<128, 128>; break;
+        default: return BRA_ERR_UNSUPPORTED;
+    }
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return BRA_ERR_CUDA;
     const cudaError_t e = launch_after_previous(kernel, dim3((unsigned)grid), dim3(threads), smem, stream, tk, tv,

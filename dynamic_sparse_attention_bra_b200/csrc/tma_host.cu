@@ -42,6 +42,21 @@ bool encode_region_map(CUtensorMap* map, const void* base, int B, int H, int W, 
               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_region_major_map(CUtensorMap* map, const void* base, int B, int H, int W, int C, int ws, int hs,
+                             int S) {
+    EncodeTiledFn fn = encoder();
+    if (!fn || H != hs * S || W != ws * S) return false;
+    // dims: channel, x in region, y in region, region column, (image, region row)
+    const cuuint64_t dims[5] = {(cuuint64_t)C, (cuuint64_t)ws, (cuuint64_t)hs, (cuuint64_t)S, (cuuint64_t)B * S};
+    const cuuint64_t strides[4] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)ws * C * 2,
+                                   (cuuint64_t)hs * W * C * 2};
+    const cuuint32_t box[5] = {32u, (cuuint32_t)ws, (cuuint32_t)hs, (cuuint32_t)S, (cuuint32_t)S};
+    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
     constexpr int kMaxDev = 64;
     static int cache[kMaxDev] = {};

@@ -14,6 +14,13 @@ namespace bra {
 bool encode_region_map(CUtensorMap* map, const void* base, int B, int H, int W, int C, int box_w,
                        int box_h, int box_c);
 
+// Tensor map over the same map viewed as (channel, x in region, y in region,
+// region column, image x region row), whose box is one head's channels of
+// every region of one image, landing region-major (region r's tokens in rows
+// r * ws * hs ... in their in-region order).
+bool encode_region_major_map(CUtensorMap* map, const void* base, int B, int H, int W, int C, int ws, int hs,
+                             int S);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -365,6 +365,7 @@ FLASH_CASES = {
     "one_route": (2, 64, 64, 64, 2, 4, 1),
     "dense_k": (1, 32, 64, 64, 2, 2, 4),              # 16 x 32 regions, k = S^2
     "odd_tiles": (1, 64, 64, 96, 3, 4, 2),            # 3 heads: tiles not a multiple of the grid
+    "regions_384": (1, 48, 32, 64, 2, 2, 2),          # 24 x 16 regions: three query tiles, none shared
 }
 
 
@@ -375,10 +376,13 @@ def test_flash_kernel(name, monkeypatch):
     check_case(bi.BraShape(B, H, W, C, heads, S, topk, "bf16"), 400 + len(name), label=f"{name} [flash]")
 
 
-def test_flash_repeated_and_bad_routes(monkeypatch):
+# 256-token regions (two query tiles sharing each key block) and 128-token
+# regions (one tile per region)
+@pytest.mark.parametrize("dims", [(1, 64, 64, 64, 2, 4, 3), (1, 64, 32, 64, 2, 4, 3)], ids=["shared", "single"])
+def test_flash_repeated_and_bad_routes(dims, monkeypatch):
     import dynamic_sparse_attention_bra_b200 as bra
     monkeypatch.setenv("BRA_ATTEND_KERNEL", "flash")
-    shape = bi.BraShape(1, 64, 64, 64, 2, 4, 3, "bf16")
+    shape = bi.BraShape(*dims, "bf16")
     rng = np.random.default_rng(9)
     idx = rng.integers(0, shape.R, size=(shape.B, shape.heads, shape.R, shape.topk)).astype(np.int32)
     idx[0, 0, :3] = [[3, 3, 3], [7, 1, 7], [0, 15, 15]]
@@ -386,7 +390,7 @@ def test_flash_repeated_and_bad_routes(monkeypatch):
     assert status == bra.BRA_OK
     ref = oracle.token_attention(inp.q_f64, inp.k_f64, inp.v_f64, idx, shape.heads, shape.S)
     err = float(np.abs(o - ref).max())
-    record_margin("repeated_routes [flash]", err, TOL["bf16"])
+    record_margin(f"repeated_routes [flash, {shape.H}x{shape.W}]", err, TOL["bf16"])
     assert err <= TOL["bf16"]
     bad = idx.copy()
     bad[0, 1, 5, 2] = -3
