@@ -365,7 +365,7 @@ FLASH_CASES = {
     "one_route": (2, 64, 64, 64, 2, 4, 1),
     "dense_k": (1, 32, 64, 64, 2, 2, 4),              # 16 x 32 regions, k = S^2
     "odd_tiles": (1, 64, 64, 96, 3, 4, 2),            # 3 heads: tiles not a multiple of the grid
-    "regions_384": (1, 48, 32, 64, 2, 2, 2),          # 24 x 16 regions: three query tiles, none shared
+    "regions_384": (1, 48, 32, 64, 2, 2, 2),          # 24 x 16 regions: three query tiles per region
 }
 
 
@@ -376,9 +376,10 @@ def test_flash_kernel(name, monkeypatch):
     check_case(bi.BraShape(B, H, W, C, heads, S, topk, "bf16"), 400 + len(name), label=f"{name} [flash]")
 
 
-# 256-token regions (two query tiles sharing each key block) and 128-token
-# regions (one tile per region)
-@pytest.mark.parametrize("dims", [(1, 64, 64, 64, 2, 4, 3), (1, 64, 32, 64, 2, 4, 3)], ids=["shared", "single"])
+# 256-token regions (two query tiles and two key blocks per region) and
+# 128-token regions (one of each)
+@pytest.mark.parametrize("dims", [(1, 64, 64, 64, 2, 4, 3), (1, 64, 32, 64, 2, 4, 3)],
+                         ids=["regions_256", "regions_128"])
 def test_flash_repeated_and_bad_routes(dims, monkeypatch):
     import dynamic_sparse_attention_bra_b200 as bra
     monkeypatch.setenv("BRA_ATTEND_KERNEL", "flash")
