@@ -94,7 +94,8 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--lce", action="store_true",
-                   help="add the local context enhancement (bra_lce, seeded 5x5 depthwise weights) to every step")
+                   help="add the local context enhancement (seeded 5x5 depthwise weights) to every step: "
+                        "bra_forward_lce, the term in the attention kernel's epilogue where it covers the shape")
     p.add_argument("--qkv", action="store_true",
                    help="start every step from the feature map: fused Q/K/V projection + routing + attention")
     p.add_argument("--backward", action="store_true",
@@ -579,10 +580,13 @@ def run_ours(args):
     def forward(b):
         if args.qkv:
             bra.bra_forward_qkv(s, b["x"], w_qkv, b_qkv, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+            if args.lce:
+                bra.bra_lce(s, b["v"], lce_w, lce_b, b["o"], sp)
+        elif args.lce:
+            # the local context term in the attention kernel's epilogue where it covers the shape
+            bra.bra_forward_lce(s, b["q"], b["k"], b["v"], lce_w, lce_b, b["o"], b["idx"], b["ws"], sp)
         else:
             bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
-        if args.lce:
-            bra.bra_lce(s, b["v"], lce_w, lce_b, b["o"], sp)
 
     def step(i):
         forward(sets[i % nsets])
@@ -722,7 +726,7 @@ def run_ours(args):
             },
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": (4 if args.lce else 3) * args.steps,
+            "gpu_launches": (4 if args.lce and args.qkv else 3) * args.steps,
             "clocks": clocks.report(),
         }
         if per_workload:

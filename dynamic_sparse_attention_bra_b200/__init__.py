@@ -26,7 +26,7 @@ __all__ = [
     "BraError", "BraShape", "shape_for", "bra_workspace_bytes", "bra_route", "bra_attend",
     "bra_forward", "bra_device_status", "bra_status_string", "forward", "library_path",
     "bra_route_noalloc", "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward",
-    "bra_qkv_project", "bra_forward_qkv", "EXPORTED_SYMBOLS",
+    "bra_qkv_project", "bra_forward_qkv", "bra_forward_lce", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,7 @@ BRA_DTYPE_F32, BRA_DTYPE_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("bra_workspace_bytes", "bra_route", "bra_attend", "bra_forward",
                     "bra_device_status", "bra_status_string", "bra_version", "bra_route_noalloc",
                     "bra_lce", "bra_selftest_bounded_wait", "bra_attend_backward", "bra_qkv_project",
-                    "bra_forward_qkv")
+                    "bra_forward_qkv", "bra_forward_lce")
 NOALLOC_MAX_MEANS = 1 << 20  # BRA_NOALLOC_MAX_MEANS
 
 
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
     lib.bra_attend.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_lce.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.bra_forward_lce.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_selftest_bounded_wait.argtypes = [sp, vp, ctypes.c_uint, ctypes.c_int, vp]
     lib.bra_attend_backward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.bra_qkv_project.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -168,6 +169,13 @@ def bra_lce(shape: BraShape, v, weight, bias, o, stream=None) -> None:
     """o += bias + 5x5 depthwise filter of v (weight fp32 [C, 5, 5], bias fp32 [C] or None)."""
     _check(_lib.bra_lce(ctypes.byref(shape), _ptr(v), _ptr(weight), _ptr(bias) if bias is not None else None,
                         _ptr(o), _stream(stream)), "bra_lce")
+
+
+def bra_forward_lce(shape: BraShape, q, k, v, weight, bias, o, idx, workspace, stream=None) -> None:
+    """Routing, attention and the local context term (weight [C,5,5] fp32, bias [C] or None) in one call."""
+    _check(_lib.bra_forward_lce(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(weight),
+                                _ptr(bias) if bias is not None else None, _ptr(o), _ptr(idx), _ptr(workspace),
+                                _stream(stream)), "bra_forward_lce")
 
 
 def bra_route_noalloc(shape: BraShape, q, k, idx, stream=None) -> None:

@@ -86,7 +86,23 @@ struct StackPlan {
     uint32_t bar_off;       // offset of barriers and tile metadata
     uint32_t smem_bytes;    // dynamic shared memory requested (incl. alignment slack)
     uint32_t tmem_cols;     // nsb S buffers of N columns, rounded up to a power of two
+    // local context term in the epilogue (8 x 8 regions, head-paired, one region per half)
+    int lce;
+    uint32_t lce_w_off;     // weights [25][C] fp32 (tap-major), then bias [C]
+    uint32_t lce_off;       // per group: V halo | O tile | row flags (kLceGroupBytes)
 };
+
+// The local context term fused into the epilogue.  A tile is one 8 x 8 region
+// of a head pair (64 channels); its softmax group writes the normalised O
+// rows to shared memory, a TMA box brings the region's V with a halo of 2
+// (12 x 12 tokens x 64 channels, zero outside the map), and the group's four
+// warps apply the 5 x 5 depthwise filter: lane = channel pair, warp = two
+// output rows, the five taps of a filter row reused along the halo row.
+constexpr int kLceSide = 12;                                      // 8 + 2 * 2
+constexpr uint32_t kLceHaloBytes = kLceSide * kLceSide * 128;     // 18 KB, 128-byte token rows
+constexpr uint32_t kLceORow = 68;                                 // O tile row stride in floats
+constexpr uint32_t kLceOBytes = 64 * kLceORow * 4;                // 17 KB
+constexpr uint32_t kLceGroupBytes = kLceHaloBytes + kLceOBytes + 1024;  // + row flags
 
 struct TileMeta {
     int b, h[2];                   // batch, head of each half
@@ -104,6 +120,9 @@ struct Barriers {
     uint64_t s_full[kMaxSBuf], o_full[kMaxSBuf], s_free[kMaxSBuf];
     uint64_t p_full[4];
     uint64_t drain[2];
+    uint64_t halo_full[4];  // a group's V halo landed
+    uint64_t gsync[4];      // the 128 threads of a group meet
+    uint64_t wready;        // the filter weights are in shared memory
     TileMeta meta[kMaxStages];
     int32_t routes[kProd][kRouteAhead][32];  // per producer warp: routes of its next tiles
     uint32_t tmem;
@@ -137,11 +156,31 @@ struct RowState {
 
 // WGS softmax warp groups (1, 2 or 4); KN64: every window is exactly 64 keys;
 // CP: compact P with one P V accumulator per query region.
-template <int WGS, bool KN64, bool CP>
+// Two fp32 lanes in one 64-bit register (x in the low half); fma.rn.f32x2
+// multiplies and adds both, each rounded as fmaf would.
+__device__ __forceinline__ uint64_t lce_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void lce_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t lce_fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// LCE: the local context term in the epilogue (th: V halo boxes; lce_weight,
+// lce_bias: the filter's weights [C][5][5] and bias [C] or null).
+template <int WGS, bool KN64, bool CP, bool LCE>
 __global__ void __launch_bounds__(32 * kCtrl + 128 * WGS, 1)
 bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, const int32_t* __restrict__ idx,
-                        __nv_bfloat16* __restrict__ o, Geometry g, StackPlan p, int* status) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap th,
+                        const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ o,
+                        const float* __restrict__ lce_weight, const float* __restrict__ lce_bias, Geometry g,
+                        StackPlan p, int* status) {
     constexpr int kThreads = 32 * kCtrl + 128 * WGS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -165,6 +204,13 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
         for (int b = 0; b < p.np; ++b) ptx::mbar_init(&sb->p_full[b], 128);
         ptx::mbar_init(&sb->drain[0], 1);
         ptx::mbar_init(&sb->drain[1], 1);
+        if (LCE) {
+            for (int x = 0; x < WGS; ++x) {
+                ptx::mbar_init(&sb->halo_full[x], 1);
+                ptx::mbar_init(&sb->gsync[x], 128);
+            }
+            ptx::mbar_init(&sb->wready, 128 * WGS);
+        }
         sb->abort = 0;
         ptx::mbar_init_fence();
     }
@@ -189,7 +235,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
     }
     // A tile of bf16 ones (same shape as one V half): P times it gives every
     // row's sum of P on the tensor core.
-    for (uint32_t i = p.ones_off / 16 + threadIdx.x; i < p.bar_off / 16; i += kThreads)
+    for (uint32_t i = p.ones_off / 16 + threadIdx.x; i < p.lce_w_off / 16; i += kThreads)
         reinterpret_cast<uint4*>(smem)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     ptx::fence_proxy_async_smem();
     __syncthreads();
@@ -433,6 +479,29 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
         const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
         const uint32_t full_live = g.topk >= 32 ? 0xffffffffu : ((1u << g.topk) - 1u);
         const float sl = kLog2e * rsqrtf(32.f);
+        // local context term: the filter in shared memory, tap-major ([25][C]
+        // fp32, then the bias), staged once by all softmax threads
+        float* lce_w = reinterpret_cast<float*>(smem + p.lce_w_off);
+        uint8_t* lce_grp = smem + p.lce_off + (uint32_t)wg * kLceGroupBytes;  // halo | O tile | flags
+        float* lce_o = reinterpret_cast<float*>(lce_grp + kLceHaloBytes);
+        uint8_t* lce_ok = lce_grp + kLceHaloBytes + kLceOBytes;  // [token][half]: the row was written
+        uint32_t gsync_phase = 0, halo_phase = 0, halo_issued = 0;
+        bool lce_failed = false;
+        // the group's 128 threads meet (bounded wait; false once the kernel aborts)
+        auto group_sync = [&]() -> bool {
+            ptx::mbar_arrive(&sb->gsync[wg]);
+            return wait_or_abort(&sb->gsync[wg], (gsync_phase++) & 1, sb, status);
+        };
+        if (LCE) {
+            const int n_st = 128 * WGS, st_i = (int)threadIdx.x - 32 * kCtrl;
+            for (int x = st_i; x < 25 * g.C; x += n_st) {
+                const int tap = x / g.C, c = x - tap * g.C;
+                lce_w[x] = __ldg(lce_weight + c * 25 + tap);
+            }
+            for (int c = st_i; c < g.C; c += n_st) lce_w[25 * g.C + c] = lce_bias ? __ldg(lce_bias + c) : 0.f;
+            ptx::mbar_arrive(&sb->wready);
+            if (!wait_or_abort(&sb->wready, 0, sb, status)) lce_failed = true;
+        }
 
         // O = (P V) / l for tile j, then release its TMEM buffer.
         auto epilogue = [&](int j, const RowState& st) -> bool {
@@ -451,6 +520,27 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             const float l = __uint_as_float(lw);
             const bool write = st.region >= 0 && l > 0.f;
             const float inv = write ? 1.f / l : 0.f;
+            if (LCE) {
+                // the normalised row (fp32) into the group's O tile; the local
+                // context term is added and O stored once, after the whole tile
+                float* orow = lce_o + (uint32_t)tok * kLceORow + (uint32_t)half * 32u;
+#pragma unroll
+                for (int h16 = 0; h16 < 2; ++h16) {
+                    if (h16 == 1) {
+                        ptx::tmem_ld16(tmem + lane_addr + o_col + 16, r);
+                        ptx::tmem_wait16(r);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<float4*>(orow + 16 * h16 + 4 * c) =
+                            make_float4(__uint_as_float(r[4 * c]) * inv, __uint_as_float(r[4 * c + 1]) * inv,
+                                        __uint_as_float(r[4 * c + 2]) * inv, __uint_as_float(r[4 * c + 3]) * inv);
+                }
+                lce_ok[tok * 2 + half] = write ? 1 : 0;
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&sb->s_free[sbuf]);
+                return true;
+            }
             const size_t ooff = write ? token_offset(g, st.b, st.region, tok) + (size_t)st.h * 32 : 0;
             int4* dst = write && in_bounds(ooff + 31, map_elems(g), status) ? reinterpret_cast<int4*>(o + ooff) : nullptr;
 #pragma unroll
@@ -476,11 +566,84 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             return true;
         };
 
+        // Local context term of tile i (one 8 x 8 region, 64 channels) once its
+        // O rows are in the group's O tile: lane = channel pair, this warp's
+        // output rows 2q and 2q + 1; halo rows 2q .. 2q + 5 each feed the
+        // output rows they are within two rows of, five taps per filter row.
+        auto lce_phase = [&](int i) -> bool {
+            if (!group_sync()) return false;  // every O row of the tile is in shared memory
+            if (!wait_or_abort(&sb->halo_full[wg], (halo_phase++) & 1, sb, status)) return false;
+            const int t = blockIdx.x + i * gridDim.x;
+            const int u = t / p.tiles_bh, r = t - u * p.tiles_bh;
+            const int b = u / (g.heads / 2), hd0 = 2 * (u - b * (g.heads / 2));
+            const int ri = r / g.S, rj = r - ri * g.S;
+            const int c0 = hd0 * 32 + 2 * lane;  // this lane's channels c0, c0 + 1
+            uint64_t acc[2][8];
+            {
+                const float2 bias = *reinterpret_cast<const float2*>(lce_w + 25 * g.C + c0);
+#pragma unroll
+                for (int orow = 0; orow < 2; ++orow)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) {
+                        const float2 ov =
+                            *reinterpret_cast<const float2*>(lce_o + (uint32_t)((2 * q + orow) * 8 + x) * kLceORow + 2 * lane);
+                        acc[orow][x] = lce_pack(ov.x + bias.x, ov.y + bias.y);
+                    }
+            }
+#pragma unroll
+            for (int hr = 0; hr < 6; ++hr) {
+                const uint8_t* hrow = lce_grp + (uint32_t)(2 * q + hr) * (kLceSide * 128u) + 4u * lane;
+                uint64_t hv[kLceSide];
+#pragma unroll
+                for (int hx = 0; hx < kLceSide; ++hx) {
+                    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(hrow + hx * 128);
+                    hv[hx] = lce_pack(__uint_as_float(w2 << 16), __uint_as_float(w2 & 0xffff0000u));
+                }
+#pragma unroll
+                for (int orow = 0; orow < 2; ++orow) {
+                    const int dy = hr - orow;  // filter row applied to this halo row for output row 2q + orow
+                    if (dy < 0 || dy > 4) continue;
+                    uint64_t wv[5];
+#pragma unroll
+                    for (int dx = 0; dx < 5; ++dx)
+                        wv[dx] = *reinterpret_cast<const uint64_t*>(lce_w + (dy * 5 + dx) * g.C + c0);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+#pragma unroll
+                        for (int dx = 0; dx < 5; ++dx) acc[orow][x] = lce_fma2(wv[dx], hv[x + dx], acc[orow][x]);
+                }
+            }
+#pragma unroll
+            for (int orow = 0; orow < 2; ++orow)
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const int tk = (2 * q + orow) * 8 + x;
+                    if (!lce_ok[tk * 2 + (lane >> 4)]) continue;  // the attention row was not written
+                    const size_t off = (((size_t)b * g.H + ri * 8 + 2 * q + orow) * g.W + rj * 8 + x) * g.C + c0;
+                    if (!in_bounds(off + 1, map_elems(g), status)) continue;
+                    float lo, hi;
+                    lce_unpack(acc[orow][x], lo, hi);
+                    *reinterpret_cast<uint32_t*>(o + off) = ptx::pack_bf16x2(lo, hi);
+                }
+            return group_sync();  // the tile's O tile and halo are free again
+        };
+
         RowState prev = {-1, 0, 0};
-        bool ok = true;
+        bool ok = !lce_failed;
         int last = -1;
         for (int i = wg; ok && i < my_tiles; i += WGS) {
             const int s = i % p.stages, sbuf = i % p.nsb, pb = i % p.np;
+            if (LCE && q == 0 && lane == 0) {
+                // this tile's region with a halo of 2, both heads (the group's
+                // previous tile is done with the buffer: its last group_sync)
+                const int t = blockIdx.x + i * gridDim.x;
+                const int u = t / p.tiles_bh, r = t - u * p.tiles_bh;  // one region per tile
+                const int b = u / (g.heads / 2), hd0 = 2 * (u - b * (g.heads / 2));
+                const int ri = r / g.S, rj = r - ri * g.S;
+                ptx::mbar_arrive_expect_tx(&sb->halo_full[wg], kLceHaloBytes);
+                ptx::tma_load_4d(ptx::smem_addr(lce_grp), &th, hd0 * 32, rj * 8 - 2, ri * 8 - 2, b, &sb->halo_full[wg]);
+                ++halo_issued;
+            }
             if (!wait_or_abort(&sb->full[s], (i / p.stages) & 1, sb, status)) break;
             if (!wait_or_abort(&sb->s_full[sbuf], (i / p.nsb) & 1, sb, status)) break;
             ptx::tc_fence_after();
@@ -580,9 +743,14 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 last = i;
             } else {
                 ok = epilogue(i, cur);
+                if (LCE && ok) ok = lce_phase(i);
             }
         }
         if (ok && last >= 0) epilogue(last, prev);
+        // a halo load issued for a tile whose filter phase never ran must land
+        // before the CTA exits
+        if (LCE && q == 0 && lane == 0 && halo_phase < halo_issued)
+            ptx::mbar_wait(&sb->halo_full[wg], halo_phase & 1, kWait);
     }
 
     ptx::tc_fence_before();
@@ -593,8 +761,12 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
     }
 }
 
-bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
+bool make_stack_plan(const Geometry& g, int max_groups, bool lce, StackPlan* p) {
     if (g.d != 32 || g.n % 16 != 0 || g.n > 64) return false;
+    // the fused local context term: 8 x 8 regions, head pairs, one region per
+    // half, the filter of at most 128 channels in shared memory
+    if (lce && (g.ws != 8 || g.hs != 8 || g.heads % 2 != 0 || g.C > 128)) return false;
+    p->lce = lce ? 1 : 0;
     const int kn = g.topk * g.n;
     if (kn > 256 || kn % 32 != 0 || g.topk > kMaxRoutes) return false;
     p->kn = kn;
@@ -632,6 +804,8 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     // outside each row's window, which separate buffers keep from the start).
     p->pin = (p->cp || p->Gq == 1) && 2u * p->p_half <= p->v_off ? 1 : 0;
     static const int kOptions[6][3] = {{4, 1, 5}, {2, 2, 3}, {2, 1, 3}, {1, 2, 3}, {2, 1, 2}, {1, 1, 2}};
+    // the filter ([25][C] weights and the bias) and, per group, the halo, the O tile and row flags
+    const uint32_t lce_w_bytes = lce ? ((26u * (uint32_t)g.C * 4u + 1023u) & ~1023u) : 0u;
     int stages = 0;
     bool found = false;
     for (int o = 0; o < 6 && !found; ++o) {
@@ -639,11 +813,13 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
         if (kOptions[o][0] > max_groups || p->nsb % kOptions[o][0] != 0 ||
             p->nsb < kOptions[o][0] * kOptions[o][1])
             continue;
+        if (lce && (kOptions[o][1] != 1 || p->Gq != 1 || !p->hp)) continue;  // the filter phase follows each epilogue
         p->wgs = kOptions[o][0];
         p->pdepth = kOptions[o][1];
         p->np = p->wgs * p->pdepth;
         const uint32_t pbytes = p->pin ? 0u : (uint32_t)p->np * 2u * p->p_half;
-        const uint32_t used = 1024 + misc + ones_bytes + pbytes;
+        const uint32_t lce_bytes = lce ? lce_w_bytes + (uint32_t)p->wgs * kLceGroupBytes : 0u;
+        const uint32_t used = 1024 + misc + ones_bytes + pbytes + lce_bytes;
         stages = used < kSmemBudget ? (int)((kSmemBudget - used) / p->stage_bytes) : 0;
         found = stages >= kOptions[o][2] && stages >= p->wgs;
     }
@@ -652,7 +828,9 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
     p->stages = stages;
     p->p_off = (uint32_t)stages * p->stage_bytes;
     p->ones_off = p->p_off + (p->pin ? 0u : (uint32_t)p->np * 2u * p->p_half);
-    p->bar_off = p->ones_off + ones_bytes;
+    p->lce_w_off = p->ones_off + ones_bytes;
+    p->lce_off = p->lce_w_off + lce_w_bytes;
+    p->bar_off = p->lce_off + (lce ? (uint32_t)p->wgs * kLceGroupBytes : 0u);
     p->smem_bytes = p->bar_off + (uint32_t)sizeof(Barriers) + 1024;
     p->nprod = stages < kProd ? stages : kProd;
     uint32_t cols = 32;
@@ -663,42 +841,81 @@ bool make_stack_plan(const Geometry& g, int max_groups, StackPlan* p) {
 
 }  // namespace
 
-bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, const void* v,
-                               const int32_t* idx, void* o, int* status, cudaStream_t stream) {
+namespace {
+
+// One launch of the stack kernel; ``weight`` non-null selects the variant with
+// the local context term in the epilogue.
+bra_status stack_launch(const Geometry& g, const void* q, const void* k, const void* v, const float* weight,
+                        const float* bias, const int32_t* idx, void* o, int* status, cudaStream_t stream) {
     // BRA_STACK_GROUPS caps the softmax warp groups (1, 2 or 4; default 4).
     int max_groups = 4;
     if (const char* env = getenv("BRA_STACK_GROUPS")) {
         const int v = atoi(env);
         if (v >= 1 && v <= 4) max_groups = v;
     }
+    const bool lce = weight != nullptr;
     StackPlan p;
-    if (!make_stack_plan(g, max_groups, &p)) return BRA_ERR_UNSUPPORTED;
-    CUtensorMap tq, tk, tv;
+    if (!make_stack_plan(g, max_groups, lce, &p)) return BRA_ERR_UNSUPPORTED;
+    CUtensorMap tq, tk, tv, th;
     if (!encode_region_map(&tq, q, g.B, g.H, g.W, g.C, g.ws, g.hs, p.hp ? 64 : 32) ||
         !encode_region_map(&tk, k, g.B, g.H, g.W, g.C, g.ws, g.hs, 32) ||
         !encode_region_map(&tv, v, g.B, g.H, g.W, g.C, g.ws, g.hs, 32))
         return BRA_ERR_UNSUPPORTED;
+    if (lce) {
+        if (!encode_halo_map(&th, v, g.B, g.H, g.W, g.C, kLceSide, kLceSide)) return BRA_ERR_UNSUPPORTED;
+    } else {
+        th = tv;  // unused
+    }
     const int sms = sm_count();
     if (sms <= 0) return BRA_ERR_CUDA;
     const int grid = p.tiles < sms ? p.tiles : sms;
-    using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, const int32_t*, __nv_bfloat16*, Geometry,
-                              StackPlan, int*);
+    using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, const int32_t*, __nv_bfloat16*,
+                              const float*, const float*, Geometry, StackPlan, int*);
     // [cp][groups 1, 2, 4][kn == 64]
     static const KernelFn kKernels[2][3][2] = {
-        {{bra_attend_stack_kernel<1, false, false>, bra_attend_stack_kernel<1, true, false>},
-         {bra_attend_stack_kernel<2, false, false>, bra_attend_stack_kernel<2, true, false>},
-         {bra_attend_stack_kernel<4, false, false>, bra_attend_stack_kernel<4, true, false>}},
-        {{bra_attend_stack_kernel<1, false, true>, bra_attend_stack_kernel<1, true, true>},
-         {bra_attend_stack_kernel<2, false, true>, bra_attend_stack_kernel<2, true, true>},
-         {bra_attend_stack_kernel<4, false, true>, bra_attend_stack_kernel<4, true, true>}}};
-    const KernelFn kernel = kKernels[p.cp][p.wgs == 4 ? 2 : p.wgs - 1][p.kn == 64 ? 1 : 0];
+        {{bra_attend_stack_kernel<1, false, false, false>, bra_attend_stack_kernel<1, true, false, false>},
+         {bra_attend_stack_kernel<2, false, false, false>, bra_attend_stack_kernel<2, true, false, false>},
+         {bra_attend_stack_kernel<4, false, false, false>, bra_attend_stack_kernel<4, true, false, false>}},
+        {{bra_attend_stack_kernel<1, false, true, false>, bra_attend_stack_kernel<1, true, true, false>},
+         {bra_attend_stack_kernel<2, false, true, false>, bra_attend_stack_kernel<2, true, true, false>},
+         {bra_attend_stack_kernel<4, false, true, false>, bra_attend_stack_kernel<4, true, true, false>}}};
+    // with the local context term: one region per half (no compact P), one or two groups
+    static const KernelFn kLceKernels[2][2] = {
+        {bra_attend_stack_kernel<1, false, false, true>, bra_attend_stack_kernel<1, true, false, true>},
+        {bra_attend_stack_kernel<2, false, false, true>, bra_attend_stack_kernel<2, true, false, true>}};
+    KernelFn kernel;
+    if (lce) {
+        if (p.cp || p.wgs > 2) return BRA_ERR_UNSUPPORTED;
+        kernel = kLceKernels[p.wgs - 1][p.kn == 64 ? 1 : 0];
+    } else {
+        kernel = kKernels[p.cp][p.wgs == 4 ? 2 : p.wgs - 1][p.kn == 64 ? 1 : 0];
+    }
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem_bytes) !=
         cudaSuccess)
         return BRA_ERR_CUDA;
     const cudaError_t e = launch_after_previous(kernel, dim3(grid), dim3(32 * kCtrl + 128 * p.wgs), p.smem_bytes,
-                                                stream, tq, tk, tv, idx, static_cast<__nv_bfloat16*>(o), g,
-                                                p, status);
+                                                stream, tq, tk, tv, th, idx, static_cast<__nv_bfloat16*>(o), weight,
+                                                bias, g, p, status);
     return e == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+}
+
+}  // namespace
+
+bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* idx, void* o, int* status, cudaStream_t stream) {
+    return stack_launch(g, q, k, v, nullptr, nullptr, idx, o, status, stream);
+}
+
+bool attend_stack_lce_covers(const Geometry& g) {
+    StackPlan p;
+    return make_stack_plan(g, 4, true, &p) && !p.cp && p.wgs <= 2;
+}
+
+bra_status attend_stack_lce_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                                   const float* weight, const float* bias, const int32_t* idx, void* o, int* status,
+                                   cudaStream_t stream) {
+    if (!weight) return BRA_ERR_INVALID_ARG;
+    return stack_launch(g, q, k, v, weight, bias, idx, o, status, stream);
 }
 
 }  // namespace bra

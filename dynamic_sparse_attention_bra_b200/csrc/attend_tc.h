@@ -19,6 +19,14 @@ bra_status attend_tc_launch(const Geometry& g, const void* q, const void* k, con
 bra_status attend_stack_launch(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* idx, void* o, int* status, cudaStream_t stream);
 
+// The same kernel with the local context term (a 5 x 5 depthwise filter of V
+// plus bias, fp32) added in its epilogue before O is rounded and stored: 8 x 8
+// regions, an even number of heads, C <= 128.
+bool attend_stack_lce_covers(const Geometry& g);
+bra_status attend_stack_lce_launch(const Geometry& g, const void* q, const void* k, const void* v,
+                                   const float* weight, const float* bias, const int32_t* idx, void* o, int* status,
+                                   cudaStream_t stream);
+
 // Persistent variant for maps of at most 256 tokens (BiFormer stage 3): each
 // (batch, head) slice's Q, K, V in shared memory, S dense over the slice,
 // each query's softmax masked to its routed regions' keys.

@@ -209,6 +209,33 @@ bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, c
                : BRA_ERR_CUDA;
 }
 
+bra_status bra_forward_lce(const bra_shape* shape, const void* q, const void* k, const void* v, const float* weight,
+                           const float* bias, void* o, int32_t* idx, void* workspace, void* stream) {
+    Geometry g;
+    bra_status rc = make_geometry(shape, &g);
+    if (rc != BRA_OK) return rc;
+    if (!q || !k || !v || !weight || !idx || !o || !workspace) return BRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(weight) || (bias && !aligned16(bias)) ||
+        !aligned16(idx) || !aligned16(o) || !aligned16(workspace))
+        return BRA_ERR_INVALID_ARG;
+    if ((int64_t)g.H > (int64_t)65535 * 8) return BRA_ERR_UNSUPPORTED;  // as bra_lce
+    const Workspace w = carve(g, workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = route_impl(shape, g, q, k, idx, w, st);
+    if (rc != BRA_OK || g.B == 0) return rc;
+    const AttendKernel choice = attend_kernel_choice();
+    if (shape->dtype == BRA_DTYPE_BF16 && (choice == AttendKernel::kAuto || choice == AttendKernel::kStack) &&
+        attend_stack_lce_covers(g)) {
+        rc = attend_stack_lce_launch(g, q, k, v, weight, bias, idx, o, w.status, st);
+        if (rc != BRA_ERR_UNSUPPORTED) return rc;
+    }
+    // other shapes: attention, then the filter added in place
+    rc = attend_impl(shape, g, q, k, v, idx, o, w, st);
+    if (rc != BRA_OK) return rc;
+    return launch_lce(shape->dtype == BRA_DTYPE_BF16, v, weight, bias, o, g, st) == cudaSuccess ? BRA_OK
+                                                                                                 : BRA_ERR_CUDA;
+}
+
 bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void* k, const void* v,
                                const int32_t* idx, const void* grad_o, float* dq, float* dk, float* dv,
                                void* workspace, void* stream) {

@@ -21,6 +21,11 @@ bool encode_region_map(CUtensorMap* map, const void* base, int B, int H, int W, 
 bool encode_region_major_map(CUtensorMap* map, const void* base, int B, int H, int W, int C, int ws, int hs,
                              int S);
 
+// Tensor map whose box is 64 channels (a head pair) of a box_w x box_h block
+// of tokens of one image, unswizzled (128-byte token rows in shared memory);
+// boxes reaching past the map are zero-filled.
+bool encode_halo_map(CUtensorMap* map, const void* base, int B, int H, int W, int C, int box_w, int box_h);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -153,6 +153,22 @@ bra_status bra_lce(const bra_shape* shape, const void* v, const float* weight, c
                    void* stream);
 
 /*
+ * The whole path with the local context term: bra_route, then the token
+ * attention with o[b,y,x,c] = attention + bias[c] + sum_{i,j} weight[c][i][j] *
+ * v[b, y+i-2, x+j-2, c] (bra_lce's filter) formed in fp32 and rounded once
+ * (blog section 2.2 step 4, third bullet; pseudocode step 7).  For bf16 maps
+ * of 8 x 8-token regions with an even number of heads and C <= 128 the filter
+ * runs in the attention kernel's epilogue (one kernel, V's halo read by TMA,
+ * O written once); other shapes run the attention, then the filter as
+ * bra_lce does (the attention output rounded before the term is added).
+ * Arguments as for bra_forward and bra_lce; a region with an out-of-range
+ * route is reported and its outputs are not written (with the fused epilogue,
+ * neither the attention nor the filter term).  Errors: as bra_forward.
+ */
+bra_status bra_forward_lce(const bra_shape* shape, const void* q, const void* k, const void* v, const float* weight,
+                           const float* bias, void* o, int32_t* idx, void* workspace, void* stream);
+
+/*
  * Reads (synchronising ``stream``) and clears the device status block in
  * ``workspace``: BRA_OK, BRA_ERR_TIMEOUT (a bounded wait in a kernel gave up;
  * that kernel's outputs are incomplete), BRA_ERR_BAD_ROUTE or, in a library

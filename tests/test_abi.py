@@ -88,6 +88,7 @@ def test_bad_shapes_rejected_before_launch(bad, code):
     assert bra._lib.bra_attend_backward(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
     assert bra._lib.bra_qkv_project(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
     assert bra._lib.bra_forward_qkv(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == code
+    assert bra._lib.bra_forward_lce(ctypes.byref(s), p, p, p, p, p, p, p, p, None) == code
     assert bra.bra_workspace_bytes(s) == 0
 
 
@@ -134,6 +135,19 @@ def test_lce_null_and_misaligned_pointers(which):
         ptrs[which] = bad
         v, w, b, o = ptrs
         assert bra._lib.bra_lce(ctypes.byref(s), v, w, b, o, None) == bra.BRA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(8))
+def test_forward_lce_null_and_misaligned_pointers(which):
+    """q, k, v, weight, o, idx and the workspace must be non-null and 16-byte
+    aligned; bias may be null but not misaligned.  Rejected on the host."""
+    s = shp()
+    good = [1 << 20] * 8
+    for bad in ((0, (1 << 20) + 4) if which != 4 else ((1 << 20) + 4,)):
+        ptrs = list(good)
+        ptrs[which] = bad
+        q, k, v, w, b, o, idx, ws = ptrs
+        assert bra._lib.bra_forward_lce(ctypes.byref(s), q, k, v, w, b, o, idx, ws, None) == bra.BRA_ERR_INVALID_ARG
 
 
 def test_selftest_rejects_bad_arguments_before_launch():
