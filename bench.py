@@ -812,7 +812,8 @@ def run_backward(args):
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype,
         "data": "synthetic",
-        "config": {**workload_config(shape, args.workload), "gradients": "fp32", "element_bytes": es},
+        "config": {**workload_config(shape, args.workload), "gradients": "fp32", "element_bytes": es,
+                   "kernel": os.environ.get("BRA_BACKWARD_KERNEL") or "auto (tensor cores where covered)"},
         "roofline": {"kernel": "bra_attend_backward", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                      "algorithmic_bytes": min_bytes, "launch_ms": ms},

@@ -42,6 +42,7 @@
 #include "kernels.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
+#include "warp_mma.cuh"
 
 namespace bra {
 namespace {
@@ -55,25 +56,9 @@ constexpr uint32_t kMaxSliceBytes = 55u * 1024u;  // K or V of one slice; two sl
 constexpr uint32_t kWait = 1u << 22;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-// D += A B for one m16n8k16 tile (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+using wmma16::ldsm_x4;
+using wmma16::ldsm_x4_t;
+using wmma16::mma16816;
 
 // Byte address of 16-byte chunk c (0..3) of row ``row`` of a slice buffer
 // written by TMA with the 64-byte swizzle (chunk index XOR bits 7-8 of the

@@ -14,4 +14,12 @@ cudaError_t launch_attend_backward(bool bf16, const void* q, const void* k, cons
                                    const void* grad_o, float* dq, float* dk, float* dv, const Geometry& g,
                                    int* status, cudaStream_t stream);
 
+// The tensor-core backward (bf16, d = 32, regions of 16..64 tokens in steps
+// of 16, topk * n <= 128 keys, topk <= 8).  dk and dv must be zero; dq is
+// written in full (zero for a region with an out-of-range route).
+bool backward_mma_covers(const Geometry& g);
+cudaError_t launch_attend_backward_mma(const void* q, const void* k, const void* v, const int32_t* idx,
+                                       const void* grad_o, float* dq, float* dk, float* dv, const Geometry& g,
+                                       int* status, cudaStream_t stream);
+
 }  // namespace bra

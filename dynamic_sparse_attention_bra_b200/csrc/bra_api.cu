@@ -251,6 +251,20 @@ bra_status bra_attend_backward(const bra_shape* shape, const void* q, const void
     if (g.B == 0) return BRA_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
+    // BRA_BACKWARD_KERNEL pins the kernel: "mma" (tensor cores) or "simt"
+    // (CUDA cores, fp32 throughout); by default the tensor-core kernel
+    // wherever it covers the shape.
+    const char* pin = getenv("BRA_BACKWARD_KERNEL");
+    const bool want_mma = !pin || strcmp(pin, "simt") != 0;
+    if (shape->dtype == BRA_DTYPE_BF16 && want_mma && backward_mma_covers(g)) {
+        // dq is written in full by the kernel; dk and dv accumulate
+        if (cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
+            return BRA_ERR_CUDA;
+        const cudaError_t e = launch_attend_backward_mma(q, k, v, idx, grad_o, dq, dk, dv, g,
+                                                         carve(g, workspace).status, st);
+        return e == cudaSuccess ? BRA_OK : BRA_ERR_CUDA;
+    }
+    if (pin && !strcmp(pin, "mma")) return BRA_ERR_UNSUPPORTED;
     if (cudaMemsetAsync(dq, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess ||
         cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
         return BRA_ERR_CUDA;
