@@ -209,17 +209,24 @@ bra_status bra_route_noalloc(const bra_shape* shape, const void* q, const void* 
  *   dP_j = <G_t, v_j>,  D_t = sum_j P_j dP_j,  dS_j = P_j (dP_j - D_t),
  *   dQ_t = sum_j dS_j k_j / sqrt(d),  dK_j = sum_t dS_tj q_t / sqrt(d),
  *   dV_j = sum_t P_tj G_t.
- * All arithmetic is fp32; dK and dV are accumulated with fp32 atomics, so
- * their last bits may differ from run to run.
+ * bf16 maps with d = 32, regions of 16, 32, 48 or 64 tokens and at most
+ * 128 routed keys per query run on tensor cores: products accumulate in
+ * fp32, and P and dS enter them rounded once to bf16 (relative error 2^-8
+ * per term).  Other shapes run on CUDA cores in fp32 throughout.  The
+ * environment variable BRA_BACKWARD_KERNEL=simt (or =mma) pins one form.
+ * dK and dV are accumulated with fp32 atomics, so their last bits may
+ * differ from run to run.
  *   shape      as for bra_attend; regions of up to about 64 tokens with up
  *              to 256 routed keys per query fit (staging in shared memory),
- *              larger ones return BRA_ERR_UNSUPPORTED
+ *              larger ones return BRA_ERR_UNSUPPORTED (as does the =mma pin
+ *              on a shape the tensor-core form does not cover)
  *   q, k, v    device, [B, H, W, C] of ``shape->dtype``, read only
  *   idx        device int32 [B, heads, S*S, topk], read only; an entry
  *              outside [0, S*S) makes the kernel skip that region's
  *              gradients and record BRA_ERR_BAD_ROUTE in the status block
  *   grad_o     device, [B, H, W, C] of ``shape->dtype``: dL/dO, read only
- *   dq, dk, dv device fp32 [B, H, W, C], written (cleared first)
+ *   dq, dk, dv device fp32 [B, H, W, C], every element written (dk, dv
+ *              cleared first, then accumulated)
  *   workspace  as for bra_attend (only its status block is used)
  * All pointers 16-byte aligned.  Errors: as bra_attend.  Allocates nothing.
  */
