@@ -378,8 +378,7 @@ bra_attend_flash_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                         uint32_t packed[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            packed[e] = on ? ptx::ex2_bf16x2(ptx::pack_bf16x2(fmaf(__uint_as_float(r[cc][2 * e]), sl, -m_new),
-                                                                                fmaf(__uint_as_float(r[cc][2 * e + 1]), sl, -m_new)))
+                            packed[e] = on ? ptx::pack_bf16x2(ptx::ex2(fmaf(__uint_as_float(r[cc][2 * e]), sl, -m_new)), ptx::ex2(fmaf(__uint_as_float(r[cc][2 * e + 1]), sl, -m_new)))
                                            : 0u;
                         const int c = c0 + 16 * cc;
                         const uint32_t atom = prow + (uint32_t)(c >> 6) * 16384u;

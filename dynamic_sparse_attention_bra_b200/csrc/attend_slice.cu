@@ -309,7 +309,7 @@ bra_attend_slice_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                         const float x0 = ((bits >> (2 * e)) & 1u) ? fmaf(__uint_as_float(r[2 * e]), sl, -msl) : -INFINITY;
                         const float x1 =
                             ((bits >> (2 * e + 1)) & 1u) ? fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl) : -INFINITY;
-                        packed[e] = ptx::ex2_bf16x2(ptx::pack_bf16x2(x0, x1));
+                        packed[e] = ptx::pack_bf16x2(ptx::ex2(x0), ptx::ex2(x1));
                     }
                     const uint32_t atom = prow + (uint32_t)(c >> 2) * 16384u;
 #pragma unroll

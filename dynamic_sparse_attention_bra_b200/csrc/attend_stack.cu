@@ -687,8 +687,8 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                     }
                     const float msl = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl;
-                    // p = 2^(s * sl - max) on bf16 pairs: P enters the MMA as bf16
-                    // anyway, and the row sums come from the same bf16 values (P x ones).
+                    // p = 2^(s * sl - max) in fp32, rounded once to bf16: P enters the
+                    // MMA as bf16, and the row sums come from the same bf16 values (P x ones).
 #pragma unroll
                     for (int c = 0; c < 64; c += 16) {
                         uint32_t r[16];
@@ -697,8 +697,7 @@ bra_attend_stack_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                         uint32_t packed[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            packed[e] = ptx::ex2_bf16x2(ptx::pack_bf16x2(fmaf(__uint_as_float(r[2 * e]), sl, -msl),
-                                                                         fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)));
+                            packed[e] = ptx::pack_bf16x2(ptx::ex2(fmaf(__uint_as_float(r[2 * e]), sl, -msl)), ptx::ex2(fmaf(__uint_as_float(r[2 * e + 1]), sl, -msl)));
                         write_p16(c, packed);
                     }
                 } else {
