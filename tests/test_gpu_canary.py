@@ -100,10 +100,34 @@ def test_local_context_writes_only_its_output():
     assert bands_intact(o_buf)
 
 
-def test_backward_writes_only_its_outputs():
+def test_forward_lce_writes_only_its_outputs():
+    """bra_forward_lce (the local context term in the attention epilogue)."""
     import torch
     import dynamic_sparse_attention_bra_b200 as bra
     shape = bi.BraShape(2, 56, 56, 64, 2, 7, 1, "bf16")
+    inp = bi.make_inputs(shape, 65)
+    q, k, v = device_inputs(inp)
+    s = bra.shape_for(*[getattr(shape, f) for f in "B H W C heads S topk".split()], "bf16")
+    ws_buf, ws = guarded((bra.bra_workspace_bytes(s),), torch.uint8)
+    ws.zero_()
+    rng = np.random.default_rng(66)
+    wt = torch.from_numpy((rng.standard_normal((shape.C, 5, 5)) / 5).astype(np.float32)).cuda()
+    bias = torch.from_numpy(rng.standard_normal(shape.C).astype(np.float32)).cuda()
+    o_buf, o = guarded(tuple(q.shape), torch.bfloat16)
+    idx_buf, idx = guarded((shape.B, shape.heads, shape.R, shape.topk), torch.int32)
+    bra.bra_forward_lce(s, q, k, v, wt, bias, o, idx, ws)
+    assert bra.bra_device_status(s, ws) == bra.BRA_OK
+    assert all(bands_intact(buf) for buf in (o_buf, idx_buf, ws_buf))
+
+
+@pytest.mark.parametrize("kernel,dims", [("mma", (2, 56, 56, 64, 2, 7, 1)), ("mma", (2, 28, 28, 128, 4, 7, 4)),
+                                         ("simt", (2, 56, 56, 64, 2, 7, 1))],
+                         ids=["mma_stage1", "mma_stage2", "simt_stage1"])
+def test_backward_writes_only_its_outputs(kernel, dims, monkeypatch):
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    monkeypatch.setenv("BRA_BACKWARD_KERNEL", kernel)
+    shape = bi.BraShape(*dims, "bf16")
     inp = bi.make_inputs(shape, 64)
     q, k, v = device_inputs(inp)
     s = bra.shape_for(*[getattr(shape, f) for f in "B H W C heads S topk".split()], "bf16")

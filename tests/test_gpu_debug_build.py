@@ -1,7 +1,8 @@
 """The debug build of the library (compiled with -DBRA_DEBUG) checks the output
 index of every attention-kernel store against its buffer and reports a miss as
 BRA_ERR_BOUNDS instead of writing.  This runs one case per attention kernel,
-at the shapes each kernel covers, through that build in a child process (the
+at the shapes each kernel covers, plus the attention with the local context
+term and the tensor-core backward, through that build in a child process (the
 package loads the build named by BRA_LIBRARY), and requires BRA_OK together
 with parity against the oracle: no kernel computes an index outside its
 output on these inputs."""
@@ -38,6 +39,22 @@ for kernel, dims in cases:
     os.environ["BRA_ATTEND_KERNEL"] = kernel
     err, rep = check_case(bi.BraShape(*dims), 77)  # asserts BRA_OK and parity
     print(kernel, dims, "ok", f"{err:.2e}")
+os.environ.pop("BRA_ATTEND_KERNEL")
+# the local context term in the stack kernel's epilogue (asserts BRA_OK and parity)
+from test_gpu_forward_lce import check_forward_lce
+check_forward_lce(bi.BraShape(2, 56, 56, 64, 2, 7, 1, "bf16"), 78, "debug build [fused lce]")
+print("fused lce", "ok")
+# the tensor-core backward (asserts BRA_OK and parity within its bound)
+import test_gpu_backward as tb
+class Env:
+    def setenv(self, k, v): os.environ[k] = v
+    def delenv(self, k, raising=True): os.environ.pop(k, None)
+for dims in ((2, 56, 56, 64, 2, 7, 1), (2, 28, 28, 128, 4, 7, 4)):
+    shape = bi.BraShape(*dims, "bf16")
+    status, got, ref, (inp, idx, g64) = tb.run(shape, 79, "mma", Env())
+    assert status == bra.BRA_OK, status
+    tb.check(shape, got, ref, "mma", "debug build", tb.mma_bounds(shape, inp, idx, g64))
+    print("backward mma", dims, "ok")
 """
 
 
@@ -47,4 +64,4 @@ def test_debug_build_reports_no_out_of_bounds_index():
     env = dict(os.environ, BRA_LIBRARY=lib)
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
-    assert r.stdout.count(" ok ") == 9, r.stdout
+    assert r.stdout.count(" ok") == 12, r.stdout
