@@ -49,7 +49,9 @@ __host__ __device__ constexpr uint32_t p_row_bytes(int kn) { return 2u * (uint32
 
 // KN: keys per query region with every route live (topk * n), a multiple of 16, <= 128.
 template <int KN>
-__global__ void __launch_bounds__(32 * kWarps)
+// Five CTAs per SM (96 registers a thread, a few spilled; the shared-memory
+// carveout set to its maximum): 20 warps instead of 16, measured 3-8 % faster.
+__global__ void __launch_bounds__(32 * kWarps, 5)
 bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx,
                                const __nv_bfloat16* __restrict__ go, float* __restrict__ dq,
@@ -344,6 +346,8 @@ cudaError_t launch_attend_backward_mma(const void* q, const void* k, const void*
     if (!kern) return cudaErrorInvalidValue;
     const size_t smem = mma_smem_bytes(g);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return cudaGetLastError();
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
         return cudaGetLastError();
     kern<<<dim3((unsigned)g.R, (unsigned)(g.B * g.heads)), 32 * kWarps, smem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
