@@ -48,9 +48,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 __host__ __device__ constexpr uint32_t p_row_bytes(int kn) { return 2u * (uint32_t)kn + 16u; }
 
 // KN: keys per query region with every route live (topk * n), a multiple of 16, <= 128.
-template <int KN>
 // Five CTAs per SM (96 registers a thread, a few spilled; the shared-memory
 // carveout set to its maximum): 20 warps instead of 16, measured 3-8 % faster.
+template <int KN>
 __global__ void __launch_bounds__(32 * kWarps, 5)
 bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx,
