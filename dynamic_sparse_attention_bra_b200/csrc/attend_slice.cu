@@ -19,7 +19,10 @@
 // are skipped.
 //
 // Roles (one CTA per SM, slices strided by the grid):
-//   warp 0     producer: the slice's Q, K, V boxes into a two-stage ring;
+//   warp 0     producer: the slice's Q, K, V boxes into a two-stage ring,
+//              then, while they land, each query region's key mask (lane per
+//              region: the OR of its routed regions' token bits) into the
+//              stage's mask buffer, so the softmax threads read a finished mask;
 //   warp 1     issues S = Q K^T for each 128-query unit of a slice;
 //   warp 2     issues O = P V (with the row sums of P) for each unit;
 //   two softmax warp groups, units alternating between them, one query row
@@ -62,12 +65,15 @@ struct SlicePlan {
     uint32_t p_bytes;       // ceil(Np / 64) atom columns of 128 rows x 128 B
     uint32_t ones_off;      // 16 rows x 64 B of bf16 ones
     uint32_t tok_off;       // R x words of uint32: the tokens of each region as key bits
+    int pre_mask;           // 1: the producer builds each query region's key mask per stage
+    uint32_t mask_off;      // per stage: R x words of uint32 (pre_mask)
+    uint32_t mask_bytes;    // R * words * 4 rounded up to 16
     uint32_t bar_off;
     uint32_t smem_bytes;
 };
 
 struct Barriers {
-    uint64_t full[kStages];   // the slice's boxes landed
+    uint64_t full[kStages];   // the slice's boxes landed (and its masks are written)
     uint64_t empty[kStages];  // the slice's last P V is done: stage free
     uint64_t s_full[kGroups], o_full[kGroups], s_free[kGroups], p_full[kGroups];
     uint64_t drain[2];
@@ -109,7 +115,7 @@ bra_attend_slice_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(&sb->full[s], 1);
+            ptx::mbar_init(&sb->full[s], p.pre_mask ? 1 + 32 : 1);  // + each producer lane's masks
             ptx::mbar_init(&sb->empty[s], 1);
         }
         for (int b = 0; b < kGroups; ++b) {
@@ -176,6 +182,34 @@ bra_attend_slice_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 const CUtensorMap* map = lane == 0 ? &tq : (lane == 1 ? &tk : &tv);
                 const uint32_t off = lane == 0 ? 0u : (lane == 1 ? p.k_off : p.v_off);
                 ptx::tma_load_4d(stage + off, map, hd * 32, 0, 0, b, &sb->full[s]);
+            }
+            if (p.pre_mask) {
+                // the slice's key masks, lane per query region; a region with an
+                // out-of-range route gets an empty mask (l = 0: nothing written)
+                const int32_t* rsrc = idx + (size_t)bh * g.R * g.topk;
+                const uint32_t* tok = reinterpret_cast<const uint32_t*>(smem + p.tok_off);
+                uint32_t* mdst = reinterpret_cast<uint32_t*>(smem + p.mask_off + (uint32_t)s * p.mask_bytes);
+                for (int r = lane; r < g.R; r += 32) {
+                    uint32_t mk[kMaxWords];
+#pragma unroll
+                    for (int w = 0; w < kMaxWords; ++w) mk[w] = 0u;
+                    bool bad = false;
+                    for (int m = 0; m < g.topk; ++m) {
+                        const int rr = __ldg(rsrc + (size_t)r * g.topk + m);
+                        if (rr < 0 || rr >= g.R) {
+                            bad = true;
+                            continue;
+                        }
+#pragma unroll
+                        for (int w = 0; w < kMaxWords; ++w)
+                            if (w < p.words) mk[w] |= tok[rr * p.words + w];
+                    }
+                    if (bad) raise_status(status, kDevBadRoute);
+#pragma unroll
+                    for (int w = 0; w < kMaxWords; ++w)
+                        if (w < p.words) mdst[r * p.words + w] = bad ? 0u : mk[w];
+                }
+                ptx::mbar_arrive(&sb->full[s]);
             }
         }
     } else if (warp == 1) {
@@ -246,7 +280,7 @@ bra_attend_slice_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
             uint32_t mk[kMaxWords];
 #pragma unroll
             for (int w = 0; w < kMaxWords; ++w) mk[w] = 0u;
-            if (valid) {
+            if (valid && !p.pre_mask) {
                 const int32_t* rows = idx + ((size_t)bh * g.R + reg) * g.topk;
                 const uint32_t* tok = reinterpret_cast<const uint32_t*>(smem + p.tok_off);
                 bool bad = false;
@@ -275,6 +309,13 @@ bra_attend_slice_kernel(const __grid_constant__ CUtensorMap tq, const __grid_con
                 }
             }
             if (!wait_or_abort(&sb->full[s], (j / kStages) & 1, sb, status)) break;
+            if (valid && p.pre_mask) {  // the producer's mask of this query region
+                const uint32_t* msrc =
+                    reinterpret_cast<const uint32_t*>(smem + p.mask_off + (uint32_t)s * p.mask_bytes) + reg * p.words;
+#pragma unroll
+                for (int w = 0; w < kMaxWords; ++w)
+                    if (w < p.words) mk[w] = msrc[w];
+            }
             if (!wait_or_abort(&sb->s_full[buf], (u / kGroups) & 1, sb, status)) break;
             ptx::tc_fence_after();
             const uint32_t sbuf = tmem + lane_addr + (uint32_t)buf * 256u;
@@ -385,9 +426,17 @@ bool make_slice_plan(const Geometry& g, SlicePlan* p) {
     p->p_bytes = (uint32_t)((p->Np + 63) / 64) * 16384u;
     p->ones_off = p->p_off + kGroups * p->p_bytes;
     p->tok_off = p->ones_off + 1024;
-    p->bar_off = p->tok_off + ((uint32_t)g.R * p->words * 4u + 15) / 16 * 16;
-    p->smem_bytes = p->bar_off + (uint32_t)sizeof(Barriers) + 1024;
-    return p->smem_bytes <= kSmemBudget;
+    p->mask_off = p->tok_off + ((uint32_t)g.R * p->words * 4u + 15) / 16 * 16;
+    p->mask_bytes = ((uint32_t)g.R * p->words * 4u + 15) / 16 * 16;
+    // the producer-built masks where two stages of them fit, else each softmax
+    // thread builds its own from the routes in global memory
+    for (int pre = 1; pre >= 0; --pre) {
+        p->pre_mask = pre;
+        p->bar_off = p->mask_off + (pre ? kStages * p->mask_bytes : 0u);
+        p->smem_bytes = p->bar_off + (uint32_t)sizeof(Barriers) + 1024;
+        if (p->smem_bytes <= kSmemBudget) return true;
+    }
+    return false;
 }
 
 }  // namespace

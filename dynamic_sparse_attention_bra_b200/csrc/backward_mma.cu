@@ -7,20 +7,23 @@
 //   dk_j += dS_j q_t / sqrt(d),  dv_j += P_j g_t,  g = dL/dO.
 //
 // bf16 maps, d = 32, regions of 16, 32, 48 or 64 tokens, at most 128 routed
-// keys per query.  One CTA of four warps per (query region, batch x head):
+// keys per query.  A team works on one (query region, batch x head): the
+// CTA's four warps together for regions of 32 tokens or more, one warp alone
+// for 16-token regions (four regions per CTA, each warp with its own slice
+// of shared memory, so that no warp idles in phase A).  Per team:
 //   staging  Q and G of the region and K, V of its topk route slots (a slot
 //            whose region repeats an earlier one is zero-filled and masked)
 //            land in shared memory by 16-byte cp.async, 80-byte token rows
 //            (64 bytes of the head + 16 of padding, so that the eight rows an
 //            ldmatrix reads fall in distinct banks);
-//   phase A  warp w takes queries 16 w .. 16 w + 15: S = Q K^T and dP = G V^T
+//   phase A  the team's warp w takes queries 16 w .. 16 w + 15: S = Q K^T and dP = G V^T
 //            as m16n8k16 tiles, the softmax and D_t with quad shuffles (rows
 //            live in the four lanes of a fragment group), dS = P (dP - D);
 //            P and dS go to shared memory as bf16 (query rows padded by 16
 //            bytes for the same reason), and dq = dS K / sqrt(d) is written
 //            straight to global memory (every query of the region is this
 //            CTA's);
-//   phase B  warp w takes key tiles 16 w', w' = w, w + 4, ...: dV = P^T G and
+//   phase B  the team's warp w takes key tiles 16 w', w' = w, w + 4, ...: dV = P^T G and
 //            dK = dS^T Q / sqrt(d) over the region's queries, the transposed
 //            operands read by ldmatrix.trans, then added to dk, dv with
 //            16-byte fp32 atomics (other query regions may route to the same
@@ -48,9 +51,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 __host__ __device__ constexpr uint32_t p_row_bytes(int kn) { return 2u * (uint32_t)kn + 16u; }
 
 // KN: keys per query region with every route live (topk * n), a multiple of 16, <= 128.
+// TW: warps per team (4: one region per CTA; 1: one region per warp, n = 16).
 // Five CTAs per SM (96 registers a thread, a few spilled; the shared-memory
 // carveout set to its maximum): 20 warps instead of 16, measured 3-8 % faster.
-template <int KN>
+template <int KN, int TW>
 __global__ void __launch_bounds__(32 * kWarps, 5)
 bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ idx,
@@ -58,14 +62,27 @@ bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
                                float* __restrict__ dk, float* __restrict__ dv, Geometry g, int* status) {
     constexpr int NT = KN / 8;  // 8-key column tiles of S
     constexpr uint32_t kPRow = p_row_bytes(KN);
+    constexpr int kTeams = kWarps / TW, kTeamThreads = 32 * TW;
     extern __shared__ __align__(16) uint8_t bwd_smem[];
-    __shared__ int slot_region[kMaxSlots];
-    __shared__ uint32_t live_slots;
-    __shared__ int bad_route;
-    const int r = blockIdx.x, bh = blockIdx.y, b = bh / g.heads, h = bh - b * g.heads;
+    __shared__ int slot_regions[kTeams][kMaxSlots];
+    __shared__ uint32_t live_team[kTeams];
+    __shared__ int bad_team[kTeams];
     const int n = g.n;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t sQ = ptx::smem_addr(bwd_smem);
+    const int lane = threadIdx.x & 31, team = (threadIdx.x >> 5) / TW;
+    const int warp = (threadIdx.x >> 5) - team * TW;  // the warp's index in its team
+    const int ttid = (int)threadIdx.x - team * kTeamThreads;
+    const int r = blockIdx.x * kTeams + team, bh = blockIdx.y, b = bh / g.heads, h = bh - b * g.heads;
+    if (r >= g.R) return;  // (one-warp teams only: the last CTA's spare warps)
+    // the team's barrier: the CTA, or for one-warp teams the warp
+    auto team_sync = [&]() {
+        if constexpr (TW == 1)
+            __syncwarp();
+        else
+            __syncthreads();
+    };
+    int* slot_region = slot_regions[team];
+    const uint32_t team_bytes = (uint32_t)(2 * n + 2 * KN) * kRowBytes + 2u * (uint32_t)n * kPRow;
+    const uint32_t sQ = ptx::smem_addr(bwd_smem) + (uint32_t)team * team_bytes;
     const uint32_t sG = sQ + (uint32_t)n * kRowBytes;
     const uint32_t sK = sG + (uint32_t)n * kRowBytes;
     const uint32_t sV = sK + (uint32_t)KN * kRowBytes;
@@ -86,31 +103,31 @@ bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         const uint32_t live = __ballot_sync(0xffffffffu, lane < g.topk && !dup);
         if (lane < g.topk) slot_region[lane] = my_r;
         if (lane == 0) {
-            live_slots = live;
-            bad_route = bad != 0;
+            live_team[team] = live;
+            bad_team[team] = bad != 0;
             if (bad) raise_status(status, kDevBadRoute);
         }
     }
-    __syncthreads();
-    if (bad_route) {
+    team_sync();
+    if (bad_team[team]) {
         // this region's gradients are skipped: its dq rows are zero
-        for (int e = threadIdx.x; e < n * 8; e += 32 * kWarps) {
+        for (int e = ttid; e < n * 8; e += kTeamThreads) {
             const int t = e >> 3, c4 = e & 7;
             const size_t off = token_offset(g, b, r, t) + (size_t)h * 32 + (size_t)c4 * 4;
             if (in_bounds(off + 3, elems, status)) *reinterpret_cast<float4*>(dq + off) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
-    const uint32_t live = live_slots;
+    const uint32_t live = live_team[team];
 
     // Staging: 16-byte chunk c of token row t (4 chunks per row).
-    for (int e = threadIdx.x; e < n * 4; e += 32 * kWarps) {
+    for (int e = ttid; e < n * 4; e += kTeamThreads) {
         const int t = e >> 2, c = e & 3;
         const size_t off = token_offset(g, b, r, t) + (size_t)h * 32 + (size_t)c * 8;
         ptx::cp_async16_zfill(sQ + (uint32_t)t * kRowBytes + (uint32_t)c * 16u, q + off, 16u);
         ptx::cp_async16_zfill(sG + (uint32_t)t * kRowBytes + (uint32_t)c * 16u, go + off, 16u);
     }
-    for (int e = threadIdx.x; e < KN * 4; e += 32 * kWarps) {
+    for (int e = ttid; e < KN * 4; e += kTeamThreads) {
         const int j = e >> 2, c = e & 3, slot = j / n, t = j - slot * n;
         const bool on = (live >> slot) & 1u;
         const size_t off = on ? token_offset(g, b, slot_region[slot], t) + (size_t)h * 32 + (size_t)c * 8 : 0;
@@ -119,7 +136,7 @@ bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
     }
     ptx::cp_async_commit();
     ptx::cp_async_wait_all();
-    __syncthreads();
+    team_sync();
 
     const float scale = rsqrtf(32.f), sl = scale * kLog2e;
     const int gq = lane >> 2, tq = lane & 3;  // fragment row group, column pair
@@ -135,7 +152,7 @@ bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         if ((live >> ((8 * j) / n)) & 1u) tile_live |= 1u << j;
 
     // ---------------------------------------------------------------- phase A
-    for (int w = warp; w < n / 16; w += kWarps) {
+    for (int w = warp; w < n / 16; w += TW) {
         const int q0 = 16 * w;
         uint32_t qa[2][4], ga[2][4];
 #pragma unroll
@@ -252,13 +269,13 @@ bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
             }
         }
     }
-    __syncthreads();
+    team_sync();
 
     // ---------------------------------------------------------------- phase B
     // A = P^T (or dS^T): 16 keys x 16 queries from the query-major rows, the
     // four 8 x 8 blocks (keys 0-7 | 8-15) x (queries 0-7 | 8-15) transposed.
     const int pa_query = (lane & 7) + ((lane >> 4) & 1) * 8, pa_key = ((lane >> 3) & 1) * 8;
-    for (int mt = warp; mt < KN / 16; mt += kWarps) {
+    for (int mt = warp; mt < KN / 16; mt += TW) {
         const int slot = (16 * mt) / n;
         if (!((live >> slot) & 1u)) continue;  // a repeated route: its P and dS are zero
         float av[4][4], ak[4][4];
@@ -311,23 +328,36 @@ bra_attend_backward_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
 using BwdKernel = void (*)(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
                            const __nv_bfloat16*, float*, float*, float*, Geometry, int*);
 
-BwdKernel kernel_for(int kn) {
+// one warp per region for 16-token regions, the CTA per region otherwise
+int team_warps(const Geometry& g) { return g.n == 16 ? 1 : kWarps; }
+
+BwdKernel kernel_for(int kn, int tw) {
+    if (tw == 1) {
+        switch (kn) {
+            case 16: return bra_attend_backward_mma_kernel<16, 1>;
+            case 32: return bra_attend_backward_mma_kernel<32, 1>;
+            case 48: return bra_attend_backward_mma_kernel<48, 1>;
+            case 64: return bra_attend_backward_mma_kernel<64, 1>;
+            case 80: return bra_attend_backward_mma_kernel<80, 1>;
+            case 96: return bra_attend_backward_mma_kernel<96, 1>;
+            case 112: return bra_attend_backward_mma_kernel<112, 1>;
+            case 128: return bra_attend_backward_mma_kernel<128, 1>;
+            default: return nullptr;
+        }
+    }
     switch (kn) {
-        case 16: return bra_attend_backward_mma_kernel<16>;
-        case 32: return bra_attend_backward_mma_kernel<32>;
-        case 48: return bra_attend_backward_mma_kernel<48>;
-        case 64: return bra_attend_backward_mma_kernel<64>;
-        case 80: return bra_attend_backward_mma_kernel<80>;
-        case 96: return bra_attend_backward_mma_kernel<96>;
-        case 112: return bra_attend_backward_mma_kernel<112>;
-        case 128: return bra_attend_backward_mma_kernel<128>;
+        case 32: return bra_attend_backward_mma_kernel<32, kWarps>;
+        case 48: return bra_attend_backward_mma_kernel<48, kWarps>;
+        case 64: return bra_attend_backward_mma_kernel<64, kWarps>;
+        case 96: return bra_attend_backward_mma_kernel<96, kWarps>;
+        case 128: return bra_attend_backward_mma_kernel<128, kWarps>;
         default: return nullptr;
     }
 }
 
 size_t mma_smem_bytes(const Geometry& g) {
-    const int kn = g.topk * g.n;
-    return (size_t)(2 * g.n + 2 * kn) * kRowBytes + (size_t)2 * g.n * p_row_bytes(kn);
+    const int kn = g.topk * g.n, teams = kWarps / team_warps(g);
+    return (size_t)teams * ((size_t)(2 * g.n + 2 * kn) * kRowBytes + (size_t)2 * g.n * p_row_bytes(kn));
 }
 
 }  // namespace
@@ -335,21 +365,23 @@ size_t mma_smem_bytes(const Geometry& g) {
 bool backward_mma_covers(const Geometry& g) {
     const int kn = g.topk * g.n;
     return g.d == 32 && g.n % 16 == 0 && g.n >= 16 && g.n <= 64 && g.topk <= kMaxSlots && kn <= 128 &&
-           kernel_for(kn) != nullptr && (long long)g.B * g.heads <= 65535;
+           kernel_for(kn, team_warps(g)) != nullptr && (long long)g.B * g.heads <= 65535 &&
+           mma_smem_bytes(g) <= 227u * 1024u;
 }
 
 cudaError_t launch_attend_backward_mma(const void* q, const void* k, const void* v, const int32_t* idx,
                                        const void* grad_o, float* dq, float* dk, float* dv, const Geometry& g,
                                        int* status, cudaStream_t stream) {
     if (g.B == 0) return cudaSuccess;
-    const BwdKernel kern = kernel_for(g.topk * g.n);
+    const int tw = team_warps(g), teams = kWarps / tw;
+    const BwdKernel kern = kernel_for(g.topk * g.n, tw);
     if (!kern) return cudaErrorInvalidValue;
     const size_t smem = mma_smem_bytes(g);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return cudaGetLastError();
     if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
         return cudaGetLastError();
-    kern<<<dim3((unsigned)g.R, (unsigned)(g.B * g.heads)), 32 * kWarps, smem, stream>>>(
+    kern<<<dim3((unsigned)((g.R + teams - 1) / teams), (unsigned)(g.B * g.heads)), 32 * kWarps, smem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
         static_cast<const __nv_bfloat16*>(v), idx, static_cast<const __nv_bfloat16*>(grad_o), dq, dk, dv, g,
         status);
