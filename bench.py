@@ -10,6 +10,11 @@ synthetic inputs.  Prints one JSON line (rank 0).
 
 ``--backward`` times bra_attend_backward (dQ, dK, dV for the routing of a
 forward pass made beforehand) on the same workload and reports its own line.
+On one GPU the default line also carries ``per_workload`` (stages 2 and 3 and
+high-res: step and attention times against their rooflines) and ``extras``
+(bra_attend_backward on stages 1 and 2 against its minimal bytes, and the
+bra_forward_lce step on stage 1 beside bra_forward), all measured in the same
+process; ``--per-workload none --extras none`` leaves them out.
 
 ``--qkv`` starts every step from the feature map X instead of Q, K, V: the
 fused projection (Q, K, V and their region means in one kernel), routing on
@@ -102,6 +107,9 @@ def parse(argv=None):
                    help="time the attention gradients (bra_attend_backward) instead of the forward")
     p.add_argument("--per-workload", default="stage2,stage3,highres",
                    help="other workloads timed in the same run (comma list; 'none': none)")
+    p.add_argument("--extras", default="backward,lce",
+                   help="entry points around the path timed in the same one-GPU run, reported under "
+                        "'extras' (comma list of backward, lce; 'none': none)")
     return p.parse_args(argv)
 
 
@@ -524,6 +532,119 @@ def time_workload(name: str, steps: int, warmup: int, dev, stream) -> dict:
     }
 
 
+def time_backward(name: str, steps: int, warmup: int, dev, stream) -> dict:
+    """bra_attend_backward back to back on one workload (a single set of inputs
+    and gradients already spans more than L2 on the stage workloads): its time
+    per call against the minimal bytes (Q, K, V, dO and I^r read once, dQ, dK,
+    dV written once in fp32)."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape, seed = bi.WORKLOADS[name]
+    inp = bi.make_inputs(shape, seed)
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    q, k, v = ((torch.from_numpy(a).view(tdt) if shape.dtype == "bf16" else torch.from_numpy(a)).to(dev)
+               for a in (inp.q_store, inp.k_store, inp.v_store))
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    ws = torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device=dev)
+    idx = torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    g = torch.Generator().manual_seed(seed + 100)
+    go = torch.randn(q.shape, generator=g).to(tdt).to(dev)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    sp = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        bra.bra_forward(s, q, k, v, o, idx, ws, sp)
+        for _ in range(warmup):
+            bra.bra_attend_backward(s, q, k, v, idx, go, dq, dk, dv, ws, sp)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps):
+                bra.bra_attend_backward(s, q, k, v, idx, go, dq, dk, dv, ws, sp)
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+    st = bra.bra_device_status(s, ws, sp)
+    if st != bra.BRA_OK:
+        raise RuntimeError(f"backward {name}: device status after timing: {bra.bra_status_string(st)}")
+    ms = start.elapsed_time(end) / steps
+    cnt = byte_counts(shape)
+    min_bytes = 4 * cnt["map"] + cnt["idx"] + 3 * shape.tokens * shape.C * 4
+    peak, peak_kind = measured_peaks()
+    del q, k, v, o, go, dq, dk, dv
+    torch.cuda.empty_cache()
+    return {"workload": workload_config(shape, name)["workload"], "entry": "bra_attend_backward",
+            "kernel": os.environ.get("BRA_BACKWARD_KERNEL") or "auto (tensor cores where covered)",
+            "ms_per_call": ms, "tokens_per_s": shape.tokens / (ms * 1e-3), "bound": "hbm",
+            "min_bytes": min_bytes, "achieved_gbs": min_bytes / (ms * 1e-3) / 1e9,
+            "frac": min_bytes / (ms * 1e-3) / 1e9 / peak, "peak_kind": peak_kind,
+            "timing": "one call = clear dK, dV + the kernel; calls back to back", "steps": steps,
+            "clocks": clocks.report()}
+
+
+def time_forward_lce(name: str, steps: int, warmup: int, dev, stream) -> dict:
+    """bra_forward_lce (routing, attention and the local context term) back to
+    back on rotating input sets larger than L2, against bra_forward on the same
+    sets in the same run."""
+    import torch
+    import dynamic_sparse_attention_bra_b200 as bra
+    shape, seed = bi.WORKLOADS[name]
+    inp = bi.make_inputs(shape, seed)
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    cnt = byte_counts(shape)
+    set_bytes = 4 * cnt["map"] + cnt["idx"]
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes))
+    s = bra.shape_for(shape.B, shape.H, shape.W, shape.C, shape.heads, shape.S, shape.topk, shape.dtype)
+    base = [torch.from_numpy(a).view(tdt) if shape.dtype == "bf16" else torch.from_numpy(a)
+            for a in (inp.q_store, inp.k_store, inp.v_store)]
+    sets = []
+    for _ in range(nsets):
+        q, k, v = (t.to(dev) for t in base)
+        sets.append(dict(q=q, k=k, v=v, o=torch.empty_like(q),
+                         idx=torch.empty((shape.B, shape.heads, shape.R, shape.topk), dtype=torch.int32, device=dev),
+                         ws=torch.zeros(bra.bra_workspace_bytes(s), dtype=torch.uint8, device=dev)))
+    g = torch.Generator().manual_seed(seed + 77)
+    lce_w = (torch.randn(shape.C * 25, generator=g) / 5.0).to(dev)
+    lce_b = torch.randn(shape.C, generator=g).to(dev)
+    sp = stream.cuda_stream
+
+    def run(i, with_lce):
+        b = sets[i % nsets]
+        if with_lce:
+            bra.bra_forward_lce(s, b["q"], b["k"], b["v"], lce_w, lce_b, b["o"], b["idx"], b["ws"], sp)
+        else:
+            bra.bra_forward(s, b["q"], b["k"], b["v"], b["o"], b["idx"], b["ws"], sp)
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            run(i, True)
+            run(i, False)
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with ClockSampler(dev.index) as clocks:
+        with torch.cuda.stream(stream):
+            ev[0].record(stream)
+            for i in range(steps):
+                run(i, True)
+            ev[1].record(stream)
+            for i in range(steps):
+                run(i, False)
+            ev[2].record(stream)
+        torch.cuda.synchronize(dev)
+    for b in sets:
+        st = bra.bra_device_status(s, b["ws"], sp)
+        if st != bra.BRA_OK:
+            raise RuntimeError(f"forward_lce {name}: device status after timing: {bra.bra_status_string(st)}")
+    lce_ms, plain_ms = ev[0].elapsed_time(ev[1]) / steps, ev[1].elapsed_time(ev[2]) / steps
+    del sets
+    torch.cuda.empty_cache()
+    return {"workload": workload_config(shape, name)["workload"], "entry": "bra_forward_lce",
+            "step_ms": lce_ms, "tokens_per_s": shape.tokens / (lce_ms * 1e-3),
+            "bra_forward_step_ms": plain_ms, "added_ms": lce_ms - plain_ms, "steps": steps,
+            "l2": f"rotating {nsets} input sets ({nsets * set_bytes / 2**20:.0f} MiB)", "clocks": clocks.report()}
+
+
 def run_ours(args):
     import torch
     import dynamic_sparse_attention_bra_b200 as bra
@@ -693,6 +814,17 @@ def run_ours(args):
     if world == 1 and not args.qkv and not args.lce:
         for name in [w for w in args.per_workload.split(",") if w in bi.WORKLOADS and w != args.workload]:
             per_workload[name] = time_workload(name, args.steps, max(args.warmup, 3), dev, stream)
+    # Entry points around the path (one GPU): the gradients and the local context term.
+    extras = {}
+    if world == 1 and not args.qkv and not args.lce:
+        wanted = [e for e in args.extras.split(",") if e]
+        if "backward" in wanted:
+            for name in ("stage1", "stage2"):
+                extras[f"backward_{name}"] = time_backward(name, min(args.steps, 100), max(args.warmup, 3), dev,
+                                                           stream)
+        if "lce" in wanted:
+            extras["forward_lce_stage1"] = time_forward_lce("stage1", min(args.steps, 200), max(args.warmup, 3),
+                                                            dev, stream)
     ms_per_step = total_ms / args.steps
     tokens = shape.tokens * world
     value = whole_job_tokens_per_s(shape.tokens, world, ms_per_step)
@@ -731,6 +863,8 @@ def run_ours(args):
         }
         if per_workload:
             line["per_workload"] = per_workload
+        if extras:
+            line["extras"] = extras
         if args.qkv:
             qkv_gbs = cnt["qkv"] / (qkv_ms * 1e-3) / 1e9
             line["qkv_roofline"] = {
