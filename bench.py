@@ -62,14 +62,16 @@ DATASHEET_HBM_GBS = 7700.0  # B200 HGX nominal HBM3e bandwidth, for context besi
 # and O is still dirty in L2 when the launch ends, so the figure is below the
 # algorithmic bytes.
 TRAFFIC_RECORDS: dict[str, dict[str, float]] = {
-    # ncu --set full, bra_attend_stack_kernel<4, 1, 0>, stage 1: read 68.26 MB + write 3.83 MB
-    "attend_stack.cu": {"37bdbeac0461348046559275bff62cf569565ddf91474f947747f0c6fcb8d94f": 72.095744e6},
-    # ncu --set full, bra_attend_warp_kernel<64> (12 warps), stage 2: read 38.77 MB + write 0.06 MB
-    "attend_warp.cu": {"0d86e7003b2f7dcb5aef6e442dbeee5b83f879c4e62fdc3e26bd769a7cb8bc58": 38.835456e6},
-    # ncu --set full, bra_attend_flash_kernel, highres: read 12.64 MB + write 0 MB
-    "attend_flash.cu": {"d6305cc7bc804bc43de0a31e74b516fa158d686d14c1ddd9034c4c964b32d6d7": 12.64e6},
-    # ncu --set full, bra_attend_slice_kernel, stage 3: read 20.95 MB + write 0 MB
-    "attend_slice.cu": {"eac7cbf607005191d84ac43bf035f66cdc772598a208926b8674cd8b4c51028e": 20.947968e6},
+    # ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch on the full workload
+    # (profiles/launches_stage1.md gives the capture command; --workload selects the stage)
+    # bra_attend_stack_kernel<4, 1, 0, 0>, stage 1: read 68.26 MB + write 3.34 MB
+    "attend_stack.cu": {"de444a53e078031d53e8d08845fa6b9cf4276aaf282a799c863f3bf5acbb37f5": 71.606016e6},
+    # bra_attend_warp_kernel<64, 16>, stage 2: read 38.77 MB + write 0.03 MB
+    "attend_warp.cu": {"b2601a5bd2bf81174f856102fd86a2efe94baf181481b9015a3669adbf06094b": 38.79296e6},
+    # bra_attend_flash_kernel, highres: read 12.64 MB + write 0 MB
+    "attend_flash.cu": {"206f6bd5db0df890ea2cd549cf0ed1e6254d335d3084a26e7703259dc62f3106": 12.644352e6},
+    # bra_attend_slice_kernel, stage 3: read 20.95 MB + write 0 MB
+    "attend_slice.cu": {"03b48fd85e880febd1d5102e078efbdc822eccc63f892d74e0cd1b6921983611": 20.951552e6},
 }
 
 # The file holding each workload's attention kernel (the kernel bra_attend
@@ -83,9 +85,9 @@ KERNEL_FILE = {"stage1": "attend_stack.cu", "stage2": "attend_warp.cu", "stage3"
 # 77 MB of Q, K, V it writes is still dirty in L2 when the launch ends, so the
 # figure is below the algorithmic bytes.
 QKV_TRAFFIC_RECORDS: dict[str, float] = {
-    # ncu --set full capture of bra_qkv_kernel<1> (8 warps, next MMA under the region sums):
-    # dram read 25.76 MB + write 20.27 MB
-    "5474982f1906dccc5f9126cc3a60e458e6d92efc3665bffbef24bfaf1d6cbe60": 46.031616e6,
+    # ncu capture of bra_qkv_kernel<1> (8 warps, next MMA under the region sums):
+    # dram read 25.77 MB + write 19.11 MB
+    "672037142a2a077ac0946e1a1c68e35e52673d0180e9b89cde6dbaf09cdc2a17": 44.871424e6,
 }
 
 
