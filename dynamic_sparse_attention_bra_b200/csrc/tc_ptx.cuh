@@ -166,7 +166,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 namespace bra {
 namespace ptx {
 
-// ---- TMA (tiled tensor loads, no multicast) -----------------------------------
+// ---- TMA (tiled tensor loads into this CTA's own shared memory) -------------
 // 4-D tiled load of one box into shared memory; completion counts bytes on ``bar``.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst_smem, const void* tmap, int c0, int c1,
                                             int c2, int c3, uint64_t* bar) {
