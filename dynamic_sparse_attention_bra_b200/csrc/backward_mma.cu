@@ -16,14 +16,15 @@
 //            land in shared memory by 16-byte cp.async, 80-byte token rows
 //            (64 bytes of the head + 16 of padding, so that the eight rows an
 //            ldmatrix reads fall in distinct banks);
-//   phase A  the team's warp w takes queries 16 w .. 16 w + 15: S = Q K^T and dP = G V^T
-//            as m16n8k16 tiles, the softmax and D_t with quad shuffles (rows
-//            live in the four lanes of a fragment group), dS = P (dP - D);
-//            P and dS go to shared memory as bf16 (query rows padded by 16
-//            bytes for the same reason), and dq = dS K / sqrt(d) is written
-//            straight to global memory (every query of the region is this
-//            CTA's);
-//   phase B  the team's warp w takes key tiles 16 w', w' = w, w + 4, ...: dV = P^T G and
+//   phase A  the team's warp w takes queries 16 w .. 16 w + 15: S = Q K^T
+//            and dP = G V^T as m16n8k16 tiles, the softmax and D_t with quad
+//            shuffles (rows live in the four lanes of a fragment group),
+//            dS = P (dP - D); P and dS go to shared memory as bf16 (query rows
+//            padded by 16 bytes for the same reason), and dq = dS K / sqrt(d)
+//            is written straight to global memory (every query of the region
+//            is this team's);
+//   phase B  the team's warp w takes key tiles 16 w', w' = w, w + (warps of
+//            the team), ...: dV = P^T G and
 //            dK = dS^T Q / sqrt(d) over the region's queries, the transposed
 //            operands read by ldmatrix.trans, then added to dk, dv with
 //            16-byte fp32 atomics (other query regions may route to the same
