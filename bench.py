@@ -138,6 +138,8 @@ def byte_counts(shape: bi.BraShape) -> dict:
         "pool": 2 * m + 2 * means,
         # fused projection: X and the layer read, Q, K, V and the means written
         "qkv": 4 * m + 2 * means + 3 * shape.C * shape.C * es + 3 * shape.C * 4,
+        # attention gradients: Q, K, V, dO and I^r read, dQ, dK, dV written in fp32
+        "backward": 4 * m + idx + 3 * shape.tokens * shape.C * 4,
         # the path from X: X read, O and I^r written
         "path_min_qkv": 2 * m + idx,
     }
@@ -572,7 +574,7 @@ def time_backward(name: str, steps: int, warmup: int, dev, stream) -> dict:
         raise RuntimeError(f"backward {name}: device status after timing: {bra.bra_status_string(st)}")
     ms = start.elapsed_time(end) / steps
     cnt = byte_counts(shape)
-    min_bytes = 4 * cnt["map"] + cnt["idx"] + 3 * shape.tokens * shape.C * 4
+    min_bytes = cnt["backward"]
     peak, peak_kind = measured_peaks()
     del q, k, v, o, go, dq, dk, dv
     torch.cuda.empty_cache()
@@ -939,8 +941,7 @@ def run_backward(args):
     cnt = byte_counts(shape)
     es = 2 if shape.dtype == "bf16" else 4
     # minimal bytes: Q, K, V, dO and I^r read once, dQ, dK, dV written once in fp32
-    grad_bytes = 3 * shape.tokens * shape.C * 4
-    min_bytes = 4 * cnt["map"] + cnt["idx"] + grad_bytes
+    min_bytes = cnt["backward"]
     peak, peak_kind = measured_peaks()
     achieved = min_bytes / (ms * 1e-3) / 1e9
     line = {
