@@ -203,3 +203,18 @@ def test_projection_rejects_what_it_does_not_cover(args):
     p = 1 << 20
     assert bra._lib.bra_qkv_project(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == bra.BRA_ERR_UNSUPPORTED
     assert bra._lib.bra_forward_qkv(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None) == bra.BRA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("dims", [
+    dict(B=4, H=14, W=14, C=256, heads=8, S=7, topk=16),   # regions of 4 tokens (stage 3)
+    dict(B=2, H=128, W=128, C=64, heads=2, S=8, topk=4),   # regions of 256 tokens (high resolution)
+    dict(B=1, H=16, W=16, C=64, heads=2, S=4, topk=16),    # 256 keys per query
+], ids=["n4", "n256", "keys256"])
+def test_backward_mma_pin_rejects_uncovered_shapes_on_the_host(dims, monkeypatch):
+    """With BRA_BACKWARD_KERNEL=mma a shape the tensor-core backward does not
+    cover is refused before any CUDA call (so this runs without a GPU)."""
+    monkeypatch.setenv("BRA_BACKWARD_KERNEL", "mma")
+    s = shp(**dims)
+    p = 1 << 20
+    rc = bra._lib.bra_attend_backward(ctypes.byref(s), p, p, p, p, p, p, p, p, p, None)
+    assert rc == bra.BRA_ERR_UNSUPPORTED, rc
