@@ -14,10 +14,11 @@ kernel, with the barrier counts of its plan (a softmax group or the producer
 warp's lanes are one role; their per-thread arrivals are one arrival).  The
 configurations are the ones the kernels' plans may choose, including the
 rules the plans enforce (producer warps <= ring stages, S buffers a multiple
-of the softmax groups and at least groups x epilogue depth).  The last test
-shows that the model catches a real mistake: a "result ready" barrier pair
-shared by four softmax groups, which ended in a bounded-wait timeout on a
-B200 before it was indexed per group.
+of the softmax groups and at least groups x epilogue depth; the flash
+kernel's ring has an even number of stages).  Negative cases show that the
+model catches real mistakes: a "result ready" barrier pair shared by four
+softmax groups (which ended in a bounded-wait timeout on a B200 before it was
+indexed per group), plans the rules reject, and an odd flash ring.
 """
 import random
 
@@ -302,3 +303,108 @@ def test_warp_kernel_ring_protocol():
     for slices in (1, 2, 3, 5):
         for seed in range(60):
             run(*warp_kernel(slices, 4), seed)
+
+
+# --------------------------------------------------------------- flash kernel
+def flash_kernel(tiles, nb, stages=4):
+    """Two softmax groups on alternate tiles (group = tile & 1), each with its
+    Q buffer and two S/O buffers; K/V blocks go through one ring indexed by the
+    step number s, where the steps of a tile pair interleave the pair's blocks
+    (s = 2 nb pair + 2 b + (tile & 1)).  Steps of a missing last odd tile are
+    skipped by every role."""
+    groups = 2
+    steps = ((tiles + 1) // 2) * 2 * nb
+    bars = {}
+    for g in range(groups):
+        bars[f"q_full{g}"], bars[f"q_empty{g}"] = Bar(f"q_full{g}"), Bar(f"q_empty{g}")
+        for y in range(2):
+            for n in ("s_full", "s_free", "p_full", "o_full"):
+                bars[f"{n}{g}{y}"] = Bar(f"{n}{g}{y}")
+    for x in range(stages):
+        bars[f"kv_full{x}"], bars[f"kv_empty{x}"] = Bar(f"kv_full{x}"), Bar(f"kv_empty{x}")
+
+    def step_at(s):
+        pair, r = divmod(s, 2 * nb)
+        b, tile = r >> 1, 2 * pair + (r & 1)
+        return (tile, b) if tile < tiles else None
+
+    def producer():
+        for s in range(steps):
+            st = step_at(s)
+            if st is None:
+                continue
+            tile, b = st
+            g, use = tile & 1, tile >> 1
+            if b == 0:
+                if use > 0:
+                    yield ("wait", f"q_empty{g}", use - 1)
+                yield ("arrive", f"q_full{g}")
+            if s >= stages:
+                yield ("wait", f"kv_empty{s % stages}", s // stages - 1)
+            yield ("arrive", f"kv_full{s % stages}")
+
+    def s_issuer():
+        for s in range(steps):
+            st = step_at(s)
+            if st is None:
+                continue
+            tile, b = st
+            g, use = tile & 1, tile >> 1
+            k = use * nb + b
+            if b == 0:
+                yield ("wait", f"q_full{g}", use)
+            yield ("wait", f"kv_full{s % stages}", s // stages)
+            if k >= 2:
+                yield ("wait", f"s_free{g}{k & 1}", (k >> 1) - 1)
+            yield ("arrive", f"s_full{g}{k & 1}")
+            if b == nb - 1:
+                yield ("arrive", f"q_empty{g}")
+
+    def pv_issuer():
+        for s in range(steps):
+            st = step_at(s)
+            if st is None:
+                continue
+            tile, b = st
+            g, use = tile & 1, tile >> 1
+            k = use * nb + b
+            yield ("wait", f"p_full{g}{k & 1}", k >> 1)
+            yield ("arrive", f"o_full{g}{k & 1}")
+            yield ("arrive", f"kv_empty{s % stages}")
+
+    def softmax(g):
+        def fold(k):
+            yield ("wait", f"o_full{g}{k & 1}", k >> 1)
+            yield ("arrive", f"s_free{g}{k & 1}")
+
+        for tile in range(g, tiles, groups):
+            use = tile >> 1
+            for b in range(nb):
+                k = use * nb + b
+                yield ("wait", f"s_full{g}{k & 1}", k >> 1)
+                yield ("arrive", f"p_full{g}{k & 1}")
+                if b > 0:
+                    yield from fold(k - 1)
+            yield from fold(use * nb + nb - 1)
+
+    roles = {"producer": producer(), "s_issuer": s_issuer(), "pv_issuer": pv_issuer(),
+             "softmax0": softmax(0), "softmax1": softmax(1)}
+    return roles, bars
+
+
+@pytest.mark.parametrize("nb", [1, 2, 8])
+def test_flash_kernel_protocol(nb):
+    """Four ring stages (even, like the steps of a pair), odd and even tile counts."""
+    for tiles in (1, 2, 3, 5, 6):
+        for seed in range(40):
+            run(*flash_kernel(tiles, nb), seed)
+
+
+def test_flash_ring_needs_an_even_stage_count_with_a_missing_tile():
+    """With an odd number of stages a skipped step and a later real one can
+    share a stage (here steps +1 and +4 of the last pair, four blocks per
+    tile, three stages): the stage's phase count falls behind, and the real
+    step's load waits for a release that never comes."""
+    with pytest.raises(ProtocolError):
+        for seed in range(100):
+            run(*flash_kernel(3, 4, stages=3), seed)
